@@ -1,0 +1,171 @@
+/*
+ * helix.h -- C ABI of libhelix.so: KV-parallel (sequence-sharded) decode attention on one B200.
+ *
+ * The method ("Helix Parallelism: Rethinking Sharding Strategies for Interactive Multi-Million-Token
+ * LLM Decoding"; paper summary page, fdeinterviews.com, paragraph on KV parallelism): the KV history
+ * of every request is split along the sequence into KVP shards. For one new query token each shard
+ * attends over its own slice and returns a partial output plus the log-sum-exp (LSE) of its logits;
+ * an LSE-rescaling combine then yields exactly the full-context result. On one GPU the shards are
+ * partitions of one paged pool in HBM, and the combine reads the partials from HBM where the
+ * multi-GPU system would run an all-to-all.
+ *
+ * Three calls make one decode-attention layer step:
+ *   helix_kv_append     place the new token's K/V round-robin across shards (16-token blocks)
+ *   helix_attn_partial  per-shard partial attention -> O_partial[shard][B][Hq][dv], lse[shard][B][Hq]
+ *   helix_attn_combine  O = sum_s exp(lse_s - LSE) * O_s, LSE = log sum_s exp(lse_s)
+ *
+ * Conventions (all calls):
+ *  - Every pointer argument that names tensor data is DEVICE memory owned by the caller; the
+ *    library never allocates, frees or retains it beyond the call. Scratch space for the partial
+ *    call is a caller-provided workspace (size from helix_attn_workspace_size).
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default stream). Host-side argument
+ *    validation happens before any launch: on error the call returns a status and launches nothing.
+ *  - Conditions only the device can see (a page id outside the pool, a history longer than the
+ *    page table) set bits in the optional `*err_word` of the cache (HELIX_DEVERR_*), skip the
+ *    affected work and never trap. The caller reads err_word after synchronising.
+ *  - A failed launch returns HELIX_ERR_CUDA. No C++ exception crosses this interface.
+ *  - Tensors are dense, row-major, with the shapes given below; every base pointer must be 16-byte
+ *    aligned.
+ *  - Calls that share a workspace or a cache must be ordered on one stream (or by events).
+ */
+#ifndef HELIX_H_
+#define HELIX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared opaquely so this header needs no CUDA headers. */
+typedef struct CUstream_st* helix_stream_t;
+
+typedef enum {
+  HELIX_OK = 0,
+  HELIX_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misaligned pointer, workspace too small */
+  HELIX_ERR_UNSUPPORTED = 2, /* a shape/dtype combination no kernel is built for */
+  HELIX_ERR_CAPACITY = 3,    /* the call cannot fit its work in the sizes given */
+  HELIX_ERR_CUDA = 4,        /* a CUDA runtime error (launch failure, no device, ...) */
+  HELIX_ERR_TIMEOUT = 5      /* reserved for host-side waits with a limit */
+} helix_status;
+
+/* Bits written (OR-ed) into *err_word by the kernels. */
+#define HELIX_DEVERR_PAGE_ID 0x1u      /* page_table entry < 0 or >= num_pages: page skipped */
+#define HELIX_DEVERR_CAPACITY 0x2u     /* a local index past max_pages_per_shard pages: skipped */
+#define HELIX_DEVERR_SHARD 0x4u        /* contiguous layout placed a token past the last shard */
+#define HELIX_DEVERR_WAIT_TIMEOUT 0x8u /* an on-chip pipeline wait ran out of its limit */
+
+typedef enum { HELIX_KV_BF16 = 0, HELIX_KV_NVFP4 = 1 } helix_kv_dtype;
+typedef enum { HELIX_ATTN_GQA = 0, HELIX_ATTN_MLA = 1 } helix_attn_kind;
+typedef enum { HELIX_LAYOUT_RR = 0, HELIX_LAYOUT_CONTIG = 1 } helix_layout;
+
+/*
+ * The paged, sequence-sharded KV cache of one attention layer.
+ *
+ * Placement of history token t (0-based global position) of request b:
+ *   HELIX_LAYOUT_RR (paper summary, paragraph on the Helix layouts; NVIDIA technical blog, Korean
+ *   edition, KV-cache section, round-robin example): block j = t / rr_block goes to shard
+ *   s = j % kvp, at local index l = (j / kvp) * rr_block + t % rr_block.
+ *   HELIX_LAYOUT_CONTIG: s = t / contig_chunk, l = t % contig_chunk.
+ * Local index l is stored in page page_table[s][b][l / page_tokens] at slot l % page_tokens.
+ *
+ * Pool layouts (P = num_pages, H = num_kv_heads, T = page_tokens, d = head_dim):
+ *   GQA, BF16 : k_pool, v_pool  bf16  [P][H][T][d]
+ *   GQA, NVFP4: k_pool, v_pool  uint8 [P][H][T][d/2]   E2M1 codes, element 2i in the low nibble
+ *               k_scale, v_scale uint8 [P][H][T][d/16] E4M3 scale of elements 16j..16j+15
+ *   MLA, BF16 : k_pool          bf16  [P][T][d] with d = 576 (H = 1); V is columns [0, v_dim) of
+ *               the same rows (v_pool must be NULL): keys and values share one latent row.
+ *
+ * State updated by helix_kv_append: seq_lens[b] (history length of request b) and
+ * shard_lens[s][b] (tokens shard s holds for request b). helix_attn_partial reads shard_lens.
+ */
+typedef struct helix_kv_cache {
+  int32_t kind;                /* helix_attn_kind */
+  int32_t kv_dtype;            /* helix_kv_dtype */
+  int32_t layout;              /* helix_layout */
+  int32_t kvp;                 /* number of KV-parallel shards, >= 1 */
+  int32_t batch;               /* requests B */
+  int32_t num_kv_heads;        /* Hkv (GQA); 1 for MLA */
+  int32_t head_dim;            /* d: 64 or 128 (GQA), 576 (MLA) */
+  int32_t v_dim;               /* dv: = head_dim (GQA), 512 (MLA) */
+  int32_t page_tokens;         /* tokens per page; 64 */
+  int32_t rr_block;            /* round-robin block; 16 */
+  int32_t contig_chunk;        /* tokens per shard, HELIX_LAYOUT_CONTIG only */
+  int32_t num_pages;           /* pages in the pool */
+  int32_t max_pages_per_shard; /* third extent of page_table */
+  int32_t reserved_;
+  void* k_pool;
+  void* v_pool;
+  void* k_scale;
+  void* v_scale;
+  const int32_t* page_table; /* int32 [kvp][batch][max_pages_per_shard] */
+  int32_t* shard_lens;       /* int32 [kvp][batch] */
+  int32_t* seq_lens;         /* int32 [batch] */
+  uint32_t* err_word;        /* optional (may be NULL): HELIX_DEVERR_* bits are OR-ed in */
+} helix_kv_cache;
+
+/*
+ * Append up to n_new tokens to every request. Row j of request b's slice gets global position
+ * seq_lens[b] + j and is placed by the cache's layout rule. Afterwards seq_lens[b] grows by the
+ * number of rows appended and shard_lens[s][b] by the number of them placed on shard s.
+ *   GQA BF16 : k_new, v_new bf16 [B][n_new][H][d]; k_new_scale = v_new_scale = NULL
+ *   GQA NVFP4: k_new, v_new uint8 [B][n_new][H][d/2]; k_new_scale, v_new_scale uint8 [B][n_new][H][d/16]
+ *   MLA      : k_new bf16 [B][n_new][576]; v_new = NULL
+ *   n_valid  : optional device int32 [B]; when given, request b appends only its first
+ *              min(max(n_valid[b], 0), n_new) rows (ragged prefill). NULL = n_new rows each.
+ * The copy is bit-exact. n_new = 0 is a no-op. Device errors: HELIX_DEVERR_PAGE_ID, _CAPACITY,
+ * _SHARD (the row is not stored; the lengths still advance).
+ */
+helix_status helix_kv_append(const helix_kv_cache* cache, const void* k_new, const void* v_new,
+                             const void* k_new_scale, const void* v_new_scale, int32_t n_new,
+                             const int32_t* n_valid, helix_stream_t stream);
+
+/*
+ * Bytes of workspace helix_attn_partial needs for this cache shape on the current device.
+ * The workspace must be zero-filled once before its first use; the kernel returns it to that
+ * state, so later calls need no clearing (unless a previous call was aborted by a device error).
+ */
+helix_status helix_attn_workspace_size(const helix_kv_cache* cache, int32_t num_q_heads,
+                                       size_t* bytes);
+
+/*
+ * Per-shard partial attention for one new query token per request (paper summary, paragraph on
+ * KV parallelism: each shard attends over its slice and returns a partial output plus an LSE).
+ *   q          bf16  [B][num_q_heads][head_dim]
+ *   o_partial  fp32  [kvp][B][num_q_heads][v_dim]  O_s = softmax-weighted V over shard s's tokens,
+ *                                                  normalised over those tokens
+ *   lse        fp32  [kvp][B][num_q_heads]          natural-log LSE of shard s's scaled logits
+ * Logit of head h against token t: softmax_scale * <q[b][h], K[t][h / (num_q_heads / H)]>.
+ * A shard with no tokens gives O_s = 0 and lse = -inf.
+ * GQA: num_q_heads % H == 0 and num_q_heads / H <= 16. MLA: num_q_heads == 128.
+ */
+helix_status helix_attn_partial(const helix_kv_cache* cache, const void* q, int32_t num_q_heads,
+                                float softmax_scale, float* o_partial, float* lse, void* workspace,
+                                size_t workspace_bytes, helix_stream_t stream);
+
+/*
+ * LSE-rescaling combine (paper review, jaehun.me, "Prompt 1.3.2 -- The Secret Weapon", boxed
+ * equation, read for partials normalised per shard): for every (b, h)
+ *   M = max_s lse_s,  LSE = M + ln sum_s exp(lse_s - M),  O = sum_s exp(lse_s - LSE) * O_s.
+ * Shards with lse = -inf carry no weight; if all are -inf, O = 0 and LSE = -inf.
+ *   o_partial fp32 [kvp][batch][num_q_heads][v_dim], lse fp32 [kvp][batch][num_q_heads]
+ *   o_out     [batch][num_q_heads][v_dim], bf16 (o_dtype 0) or fp32 (o_dtype 1)
+ *   lse_out   fp32 [batch][num_q_heads], may be NULL
+ * v_dim must be a multiple of 4.
+ */
+helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads, int32_t v_dim,
+                                const float* o_partial, const float* lse, void* o_out,
+                                int32_t o_dtype, float* lse_out, helix_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* helix_status_string(helix_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t helix_version(void);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* HELIX_H_ */

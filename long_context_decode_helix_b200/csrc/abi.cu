@@ -1,0 +1,270 @@
+// abi.cu -- the extern "C" entry points of libhelix.so: argument validation, TMA descriptor
+// encoding and dispatch to the kernels. Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "helix.h"
+#include "internal.h"
+
+namespace helix {
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a pool viewed as [rows][row_elems] with 64 x box_rows boxes, 128-byte swizzle.
+bool encode_rows_map(CUtensorMap* map, void* base, CUtensorMapDataType dt, int elem_bytes,
+                     uint64_t row_elems, uint64_t rows, uint32_t box_elems, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {row_elems, rows};
+  const cuuint64_t strides[1] = {row_elems * (uint64_t)elem_bytes};
+  const cuuint32_t box[2] = {box_elems, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sm_count(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return 0;
+}
+
+int device_max_smem(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(out, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return -1;
+  return 0;
+}
+
+// Shape checks common to every call that takes a cache.
+helix_status check_cache(const helix_kv_cache* c) {
+  if (c == nullptr) return HELIX_ERR_INVALID_ARG;
+  if (c->kvp < 1 || c->batch < 1 || c->num_kv_heads < 1 || c->head_dim < 1 || c->v_dim < 1 ||
+      c->page_tokens < 1 || c->num_pages < 1 || c->max_pages_per_shard < 1)
+    return HELIX_ERR_INVALID_ARG;
+  if (c->layout == HELIX_LAYOUT_RR) {
+    if (c->rr_block < 1) return HELIX_ERR_INVALID_ARG;
+  } else if (c->layout == HELIX_LAYOUT_CONTIG) {
+    if (c->contig_chunk < 1) return HELIX_ERR_INVALID_ARG;
+  } else {
+    return HELIX_ERR_INVALID_ARG;
+  }
+  if (c->page_table == nullptr || c->shard_lens == nullptr || c->seq_lens == nullptr)
+    return HELIX_ERR_INVALID_ARG;
+  if (!aligned4(c->page_table) || !aligned4(c->shard_lens) || !aligned4(c->seq_lens) ||
+      !aligned4(c->err_word))
+    return HELIX_ERR_INVALID_ARG;
+  if (c->k_pool == nullptr || !aligned16(c->k_pool)) return HELIX_ERR_INVALID_ARG;
+  if (c->kind == HELIX_ATTN_GQA) {
+    if (c->v_pool == nullptr || !aligned16(c->v_pool)) return HELIX_ERR_INVALID_ARG;
+    if (c->v_dim != c->head_dim) return HELIX_ERR_INVALID_ARG;
+    if (c->kv_dtype == HELIX_KV_NVFP4) {
+      if (c->head_dim % 32 != 0) return HELIX_ERR_INVALID_ARG;
+      if (c->k_scale == nullptr || c->v_scale == nullptr || !aligned16(c->k_scale) ||
+          !aligned16(c->v_scale))
+        return HELIX_ERR_INVALID_ARG;
+    } else if (c->kv_dtype != HELIX_KV_BF16) {
+      return HELIX_ERR_INVALID_ARG;
+    }
+  } else if (c->kind == HELIX_ATTN_MLA) {
+    if (c->num_kv_heads != 1 || c->v_pool != nullptr || c->kv_dtype != HELIX_KV_BF16 ||
+        c->v_dim > c->head_dim)
+      return HELIX_ERR_INVALID_ARG;
+  } else {
+    return HELIX_ERR_INVALID_ARG;
+  }
+  // pool rows, local indices and prefix sums are 32-bit on the device
+  const int64_t rows = (int64_t)c->num_pages * c->num_kv_heads * c->page_tokens;
+  const int64_t units = (int64_t)c->batch * c->num_kv_heads * c->kvp;
+  if (rows > INT32_MAX || units * c->max_pages_per_shard > INT32_MAX ||
+      (int64_t)c->max_pages_per_shard * c->page_tokens > INT32_MAX)
+    return HELIX_ERR_CAPACITY;
+  return HELIX_OK;
+}
+
+struct PartialPlan {
+  int grid;
+  int units;
+  size_t ticket_bytes;
+  size_t seg_bytes;
+};
+
+helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan* plan) {
+  helix_status st = check_cache(c);
+  if (st != HELIX_OK) return st;
+  if (num_q_heads < 1 || num_q_heads % c->num_kv_heads != 0) return HELIX_ERR_INVALID_ARG;
+  if (c->kind != HELIX_ATTN_GQA) return HELIX_ERR_UNSUPPORTED;
+  if (c->page_tokens != 64) return HELIX_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return HELIX_ERR_UNSUPPORTED;
+  if (num_q_heads / c->num_kv_heads > 16) return HELIX_ERR_UNSUPPORTED;
+  if (c->kv_dtype != HELIX_KV_BF16) return HELIX_ERR_UNSUPPORTED;
+  int sms = 0, max_smem = 0;
+  if (device_sm_count(&sms) != 0 || device_max_smem(&max_smem) != 0) return HELIX_ERR_CUDA;
+  plan->units = c->batch * c->num_kv_heads * c->kvp;
+  if (gqa_partial_smem_bytes(c->head_dim, plan->units) > (size_t)max_smem)
+    return HELIX_ERR_CAPACITY;
+  plan->grid = sms;
+  plan->ticket_bytes = (((size_t)plan->units * sizeof(int32_t)) + 255) & ~size_t(255);
+  plan->seg_bytes = (size_t)plan->grid * 2 * gqa_segment_record_floats(c->head_dim) * sizeof(float);
+  return HELIX_OK;
+}
+
+}  // namespace
+}  // namespace helix
+
+using namespace helix;
+
+extern "C" {
+
+const char* helix_status_string(helix_status s) {
+  switch (s) {
+    case HELIX_OK: return "HELIX_OK";
+    case HELIX_ERR_INVALID_ARG: return "HELIX_ERR_INVALID_ARG";
+    case HELIX_ERR_UNSUPPORTED: return "HELIX_ERR_UNSUPPORTED";
+    case HELIX_ERR_CAPACITY: return "HELIX_ERR_CAPACITY";
+    case HELIX_ERR_CUDA: return "HELIX_ERR_CUDA";
+    case HELIX_ERR_TIMEOUT: return "HELIX_ERR_TIMEOUT";
+  }
+  return "HELIX_ERR_UNKNOWN";
+}
+
+int32_t helix_version(void) { return kVersion; }
+
+helix_status helix_kv_append(const helix_kv_cache* c, const void* k_new, const void* v_new,
+                             const void* k_new_scale, const void* v_new_scale, int32_t n_new,
+                             const int32_t* n_valid, helix_stream_t stream) {
+  helix_status st = check_cache(c);
+  if (st != HELIX_OK) return st;
+  if (n_new < 0) return HELIX_ERR_INVALID_ARG;
+  if (n_new == 0) return HELIX_OK;
+  AppendParams p{};
+  const int d = c->head_dim;
+  if (c->kind == HELIX_ATTN_GQA && c->kv_dtype == HELIX_KV_BF16) {
+    if (k_new == nullptr || v_new == nullptr || !aligned4(k_new) || !aligned4(v_new))
+      return HELIX_ERR_INVALID_ARG;
+    p.src[0] = (const uint8_t*)k_new; p.dst[0] = (uint8_t*)c->k_pool; p.row_bytes[0] = d * 2;
+    p.src[1] = (const uint8_t*)v_new; p.dst[1] = (uint8_t*)c->v_pool; p.row_bytes[1] = d * 2;
+  } else if (c->kind == HELIX_ATTN_GQA && c->kv_dtype == HELIX_KV_NVFP4) {
+    if (k_new == nullptr || v_new == nullptr || k_new_scale == nullptr || v_new_scale == nullptr ||
+        !aligned4(k_new) || !aligned4(v_new) || !aligned4(k_new_scale) || !aligned4(v_new_scale))
+      return HELIX_ERR_INVALID_ARG;
+    p.src[0] = (const uint8_t*)k_new; p.dst[0] = (uint8_t*)c->k_pool; p.row_bytes[0] = d / 2;
+    p.src[1] = (const uint8_t*)v_new; p.dst[1] = (uint8_t*)c->v_pool; p.row_bytes[1] = d / 2;
+    p.src[2] = (const uint8_t*)k_new_scale; p.dst[2] = (uint8_t*)c->k_scale; p.row_bytes[2] = d / 16;
+    p.src[3] = (const uint8_t*)v_new_scale; p.dst[3] = (uint8_t*)c->v_scale; p.row_bytes[3] = d / 16;
+  } else {  // MLA: one latent row per token, V aliases its first v_dim columns
+    if (k_new == nullptr || v_new != nullptr || !aligned4(k_new)) return HELIX_ERR_INVALID_ARG;
+    p.src[0] = (const uint8_t*)k_new; p.dst[0] = (uint8_t*)c->k_pool; p.row_bytes[0] = d * 2;
+  }
+  p.page_table = c->page_table;
+  p.shard_lens = c->shard_lens;
+  p.seq_lens = c->seq_lens;
+  p.err = c->err_word;
+  p.B = c->batch;
+  p.Hkv = c->num_kv_heads;
+  p.kvp = c->kvp;
+  p.layout = c->layout;
+  p.rr_block = c->rr_block;
+  p.contig_chunk = c->contig_chunk;
+  p.page_tokens = c->page_tokens;
+  p.max_pages = c->max_pages_per_shard;
+  p.num_pages = c->num_pages;
+  p.n_new = n_new;
+  if (!aligned4(n_valid)) return HELIX_ERR_INVALID_ARG;
+  p.n_valid = n_valid;
+  return append_launch(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+helix_status helix_attn_workspace_size(const helix_kv_cache* c, int32_t num_q_heads,
+                                       size_t* bytes) {
+  if (bytes == nullptr) return HELIX_ERR_INVALID_ARG;
+  PartialPlan plan;
+  helix_status st = plan_partial(c, num_q_heads, &plan);
+  if (st != HELIX_OK) return st;
+  *bytes = plan.ticket_bytes + plan.seg_bytes;
+  return HELIX_OK;
+}
+
+helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                                float softmax_scale, float* o_partial, float* lse, void* workspace,
+                                size_t workspace_bytes, helix_stream_t stream) {
+  PartialPlan plan;
+  helix_status st = plan_partial(c, num_q_heads, &plan);
+  if (st != HELIX_OK) return st;
+  if (q == nullptr || o_partial == nullptr || lse == nullptr || workspace == nullptr)
+    return HELIX_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o_partial) || !aligned4(lse) || !aligned16(workspace))
+    return HELIX_ERR_INVALID_ARG;
+  if (workspace_bytes < plan.ticket_bytes + plan.seg_bytes) return HELIX_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return HELIX_ERR_INVALID_ARG;
+
+  GqaParams p{};
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.page_table = c->page_table;
+  p.shard_lens = c->shard_lens;
+  p.o_part = o_partial;
+  p.lse = lse;
+  p.tickets = reinterpret_cast<int32_t*>(workspace);
+  p.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes);
+  p.err = c->err_word;
+  p.B = c->batch;
+  p.Hq = num_q_heads;
+  p.Hkv = c->num_kv_heads;
+  p.G = num_q_heads / c->num_kv_heads;
+  p.D = c->head_dim;
+  p.kvp = c->kvp;
+  p.max_pages = c->max_pages_per_shard;
+  p.num_pages = c->num_pages;
+  p.units = plan.units;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+  const uint64_t rows = (uint64_t)c->num_pages * c->num_kv_heads * c->page_tokens;
+  CUtensorMap tmK, tmV;
+  if (!encode_rows_map(&tmK, c->k_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c->head_dim, rows,
+                       64, 64) ||
+      !encode_rows_map(&tmV, c->v_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c->head_dim, rows,
+                       64, 64))
+    return HELIX_ERR_CUDA;
+  return gqa_partial_bf16_launch(tmK, tmV, p, plan.grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads, int32_t v_dim,
+                                const float* o_partial, const float* lse, void* o_out,
+                                int32_t o_dtype, float* lse_out, helix_stream_t stream) {
+  if (kvp < 1 || batch < 0 || num_q_heads < 0 || v_dim < 4 || v_dim % 4 != 0)
+    return HELIX_ERR_INVALID_ARG;
+  if (o_dtype != 0 && o_dtype != 1) return HELIX_ERR_INVALID_ARG;
+  if (o_partial == nullptr || lse == nullptr || o_out == nullptr) return HELIX_ERR_INVALID_ARG;
+  if (!aligned16(o_partial) || !aligned4(lse) || !aligned16(o_out) || !aligned4(lse_out))
+    return HELIX_ERR_INVALID_ARG;
+  return combine_launch(kvp, batch, num_q_heads, v_dim, o_partial, lse, o_out, o_dtype, lse_out,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

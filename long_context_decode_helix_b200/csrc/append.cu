@@ -1,0 +1,154 @@
+// append.cu -- place new K/V tokens into the sharded, paged pool.
+//
+// Placement (paper summary "Helix Parallelism ...", fdeinterviews.com, paragraph on the Helix
+// layouts; NVIDIA technical blog, Korean edition, KV-cache section, round-robin example): global
+// position t of a request lies in block j = t / rr_block, which goes to KVP shard j % kvp; inside the
+// shard the token keeps its global order, at local index (j / kvp) * rr_block + t % rr_block. The
+// contiguous layout puts t on shard t / contig_chunk at local index t % contig_chunk. Local index l
+// lives on the shard's page page_table[s][b][l / page_tokens], slot l % page_tokens.
+//
+// The copy is bit-exact (16/8/4-byte vector moves). Lengths advance after every copy of the call has
+// read the old seq_lens: in the same block when one block holds all of a request's new tokens,
+// otherwise in a second one-block kernel on the same stream.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "device_common.cuh"
+#include "internal.h"
+
+namespace helix {
+namespace {
+
+constexpr int kAppendThreads = 256;
+constexpr int kTokensPerBlock = 64;
+
+struct Placement {
+  int shard, local;
+};
+
+__device__ __forceinline__ Placement place(long long t, const AppendParams& p) {
+  Placement r;
+  if (p.layout == HELIX_LAYOUT_RR) {
+    const long long j = t / p.rr_block;
+    r.shard = (int)(j % p.kvp);
+    r.local = (int)((j / p.kvp) * p.rr_block + t % p.rr_block);
+  } else {
+    r.shard = (int)(t / p.contig_chunk);
+    r.local = (int)(t % p.contig_chunk);
+  }
+  return r;
+}
+
+// Tokens of [0, S) that the layout puts on shard s.
+__device__ __forceinline__ long long count_on_shard(long long S, int s, const AppendParams& p) {
+  if (p.layout == HELIX_LAYOUT_RR) {
+    const long long full = S / p.rr_block, rem = S % p.rr_block;
+    long long n = (full / p.kvp) * p.rr_block;
+    const long long left = full % p.kvp;
+    if (s < left) n += p.rr_block;
+    if (s == left) n += rem;
+    return n;
+  }
+  const long long lo = (long long)s * p.contig_chunk;
+  long long n = S - lo;
+  if (n < 0) n = 0;
+  if (n > p.contig_chunk) n = p.contig_chunk;
+  return n;
+}
+
+template <int VEC>
+__device__ __forceinline__ void copy_row(uint8_t* dst, const uint8_t* src, int bytes, int lane0,
+                                         int nlanes) {
+  using T = typename std::conditional<VEC == 16, uint4,
+                                      typename std::conditional<VEC == 8, uint2, uint32_t>::type>::type;
+  for (int o = lane0 * VEC; o < bytes; o += nlanes * VEC)
+    *reinterpret_cast<T*>(dst + o) = *reinterpret_cast<const T*>(src + o);
+}
+
+__device__ void copy_bytes(uint8_t* dst, const uint8_t* src, int bytes, int lane0, int nlanes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | bytes;
+  if ((a & 15) == 0) copy_row<16>(dst, src, bytes, lane0, nlanes);
+  else if ((a & 7) == 0) copy_row<8>(dst, src, bytes, lane0, nlanes);
+  else copy_row<4>(dst, src, bytes, lane0, nlanes);
+}
+
+__device__ __forceinline__ int rows_of(const AppendParams& p, int b) {
+  if (p.n_valid == nullptr) return p.n_new;
+  return min(max(p.n_valid[b], 0), p.n_new);
+}
+
+__device__ void update_lengths(const AppendParams& p, int b) {
+  const long long S_old = p.seq_lens[b];
+  const long long S_new = S_old + rows_of(p, b);
+  for (int s = 0; s < p.kvp; ++s) {
+    const long long add = count_on_shard(S_new, s, p) - count_on_shard(S_old, s, p);
+    p.shard_lens[s * p.B + b] += (int)add;
+  }
+  p.seq_lens[b] = (int)S_new;
+}
+
+// grid: (token blocks, B). One warp copies one (token, head) row set at a time.
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendParams p,
+                                                                bool update_here) {
+  const int b = blockIdx.y;
+  const long long S_old = p.seq_lens[b];
+  const int j0 = blockIdx.x * kTokensPerBlock;
+  const int j1 = min(rows_of(p, b), j0 + kTokensPerBlock);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = kAppendThreads / 32;
+  const int items = max(j1 - j0, 0) * p.Hkv;
+  for (int it = warp; it < items; it += nwarps) {
+    const int j = j0 + it / p.Hkv;
+    const int h = it % p.Hkv;
+    const long long t = S_old + j;
+    const Placement pl = place(t, p);
+    if (pl.shard >= p.kvp) {
+      if (lane == 0) raise_dev_error(p.err, HELIX_DEVERR_SHARD);
+      continue;
+    }
+    const int pi = pl.local / p.page_tokens;
+    const int slot = pl.local % p.page_tokens;
+    if (pi >= p.max_pages) {
+      if (lane == 0) raise_dev_error(p.err, HELIX_DEVERR_CAPACITY);
+      continue;
+    }
+    const int page = p.page_table[((size_t)pl.shard * p.B + b) * p.max_pages + pi];
+    if (page < 0 || page >= p.num_pages) {
+      if (lane == 0) raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
+      continue;
+    }
+    const size_t src_row = ((size_t)b * p.n_new + j) * p.Hkv + h;
+    const size_t dst_row = ((size_t)page * p.Hkv + h) * p.page_tokens + slot;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int rb = p.row_bytes[k];
+      if (rb == 0) continue;
+      copy_bytes(p.dst[k] + dst_row * rb, p.src[k] + src_row * rb, rb, lane, 32);
+    }
+  }
+  if (update_here) {
+    __syncthreads();
+    if (threadIdx.x == 0) update_lengths(p, b);
+  }
+}
+
+__global__ void append_lengths_kernel(const AppendParams p) {
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) update_lengths(p, b);
+}
+
+}  // namespace
+
+helix_status append_launch(const AppendParams& p, cudaStream_t stream) {
+  if (p.n_new == 0) return HELIX_OK;
+  const int nblk = (p.n_new + kTokensPerBlock - 1) / kTokensPerBlock;
+  const bool one_block = nblk == 1;
+  append_kernel<<<dim3(nblk, p.B), kAppendThreads, 0, stream>>>(p, one_block);
+  if (cudaGetLastError() != cudaSuccess) return HELIX_ERR_CUDA;
+  if (!one_block) {
+    append_lengths_kernel<<<1, 128, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return HELIX_ERR_CUDA;
+  }
+  return HELIX_OK;
+}
+
+}  // namespace helix

@@ -1,0 +1,555 @@
+// gqa_partial.cu -- per-shard partial decode attention for grouped-query attention, bf16 KV.
+//
+// What it computes (paper summary "Helix Parallelism: Rethinking Sharding Strategies for
+// Interactive Multi-Million-Token LLM Decoding", fdeinterviews.com, paragraph on KV parallelism):
+// for every request b, KV head k and KVP shard s, over the tokens T_s the shard holds,
+//     z_{h,t} = scale * <q_{b,h}, K_{t,k}>            for the G query heads h of KV head k
+//     O_s[h]  = sum_t e^{z_{h,t} - m} V_{t,k} / sum_t e^{z_{h,t} - m},   lse_s[h] = m + ln sum_t ...
+// The G heads of a group are the M = 16 rows of one m16n8k16 tensor-core tile, so the shard's K and V
+// rows stream from HBM exactly once for all heads that share them.
+//
+// Work decomposition ("stream-K" over pages): the (b, k, s) units are laid end to end as one list
+// of 64-token pages; each persistent CTA takes an equal contiguous range of that list, whatever the
+// per-request lengths are. A CTA that finishes a unit inside its range writes the normalised result
+// directly; a unit cut by range boundaries is written as unnormalised segments to the workspace and
+// merged by whichever CTA arrives last on the unit's ticket (an atomic counter -- nobody spins).
+//
+// CTA layout: warps 0-7 are two consumer warpgroups that take alternate pages; warp w of a group owns
+// tokens [16w, 16w+16) of its page. Warp 8 is the producer: one lane issues TMA tile loads of the
+// page's K and V rows (128-byte swizzle, 8 KiB per 64-column half) into an NSTAGE-deep ring guarded by
+// mbarriers. Softmax is online in fp32 and base 2 (scale * log2 e folded into the logits).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "device_common.cuh"
+#include "internal.h"
+
+namespace helix {
+namespace {
+
+constexpr int kPage = 64;         // tokens per page
+constexpr int kRows = 16;         // query-head rows per tile (G <= 16, zero-padded)
+constexpr int kConsumerWarps = 8; // two warpgroups
+constexpr int kGroups = 2;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kChunkBytes = kPage * 64 * 2;  // one 64-column half of a page-head: 8 KiB
+
+template <int D>
+struct GqaCfg {
+  static constexpr int NCH = D / 64;                        // 64-column halves per row
+  static constexpr int STAGE_BYTES = 2 * NCH * kChunkBytes;  // K + V of one (page, kv head)
+  static constexpr int NSTAGE = (D == 128) ? 5 : 10;
+  static constexpr int REC = kRows * (D + 2);  // floats per workspace segment record
+};
+
+struct SmemTail {
+  uint64_t full[16];
+  uint64_t empty[16];
+  float mstat[kConsumerWarps][kRows];
+  float lstat[kConsumerWarps][kRows];
+  int flag;
+  int abort_;
+};
+
+template <int D>
+__host__ __device__ constexpr size_t smem_bytes_for(int units) {
+  return 1024 /*alignment slack*/ + (size_t)GqaCfg<D>::NSTAGE * GqaCfg<D>::STAGE_BYTES +
+         (size_t)kRows * D * sizeof(float) + sizeof(SmemTail) + (size_t)(units + 1) * sizeof(int);
+}
+
+__device__ __forceinline__ long long range_begin(int c, long long W, int G) {
+  return (long long)c * W / G;
+}
+// CTA whose range holds page x (0 <= x < W), for ranges begin(c) = floor(c W / G) with G <= W.
+__device__ __forceinline__ int cta_of(long long x, long long W, int G) {
+  return (int)(((x + 1) * (long long)G - 1) / W);
+}
+
+// Warp-collective pipeline wait: lane 0 polls with a time limit, the result is broadcast.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    gqa_partial_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const GqaParams p) {
+  using Cfg = GqaCfg<D>;
+  constexpr int NCH = Cfg::NCH;
+  constexpr int NSTAGE = Cfg::NSTAGE;
+  constexpr int KSTEPS = D / 16;  // k-steps of the QK^T contraction
+  constexpr int NT = D / 8;       // n-tiles of the PV output
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  float* Obuf = reinterpret_cast<float*>(smem + (size_t)NSTAGE * Cfg::STAGE_BYTES);
+  SmemTail* tail = reinterpret_cast<SmemTail*>(Obuf + kRows * D);
+  int* pre = reinterpret_cast<int*>(tail + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int U = p.units;
+
+  // ---- per-unit page counts and their prefix sums (every CTA computes the same table) ----
+  for (int u = tid; u < U; u += kThreads) {
+    const int s = u % p.kvp;
+    const int b = (u / p.kvp) / p.Hkv;
+    int len = p.shard_lens[s * p.B + b];
+    int np = len > 0 ? (len + kPage - 1) / kPage : 0;
+    if (np > p.max_pages) {
+      if (blockIdx.x == 0) raise_dev_error(p.err, HELIX_DEVERR_CAPACITY);
+      np = p.max_pages;
+    }
+    pre[u + 1] = np;
+  }
+  for (int i = tid; i < kRows * D; i += kThreads) Obuf[i] = 0.f;
+  if (tid == 0) {
+    pre[0] = 0;
+    tail->flag = 0;
+    tail->abort_ = 0;
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&tail->full[i], 1);
+      mbar_init(&tail->empty[i], 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {  // inclusive scan of pre[1..U], 32 lanes x contiguous chunks
+    const int per = (U + 31) / 32;
+    const int lo = 1 + lane * per, hi = min(U + 1, lo + per);
+    int run = 0;
+    for (int i = lo; i < hi; ++i) run += pre[i];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int acc = incl - run;
+    for (int i = lo; i < hi; ++i) {
+      acc += pre[i];
+      pre[i] = acc;
+    }
+  }
+  __syncthreads();
+
+  const long long W = pre[U];
+  // Units with no tokens: O_s = 0, lse_s = -inf (handled round-robin by CTA index).
+  for (int u = blockIdx.x; u < U; u += gridDim.x) {
+    if (pre[u + 1] != pre[u]) continue;
+    const int s = u % p.kvp, bk = u / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
+    const size_t row0 = ((size_t)s * p.B + b) * p.Hq + (size_t)k * p.G;
+    for (int i = tid; i < p.G * D; i += kThreads) p.o_part[row0 * D + i] = 0.f;
+    for (int i = tid; i < p.G; i += kThreads) p.lse[row0 + i] = -INFINITY;
+  }
+  const int Geff = (int)min((long long)gridDim.x, W);
+  if ((int)blockIdx.x >= Geff) return;
+  const long long g_begin = range_begin(blockIdx.x, W, Geff);
+  const long long g_end = range_begin(blockIdx.x + 1, W, Geff);
+  // first unit: pre[u] <= g_begin < pre[u+1]
+  int u_first;
+  {
+    int lo = 0, hi = U;  // find the last u with pre[u] <= g_begin
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (pre[mid] <= g_begin) lo = mid; else hi = mid;
+    }
+    u_first = lo;
+    while (pre[u_first + 1] <= g_begin) ++u_first;
+  }
+
+  // ======================================= producer =============================================
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      int u = u_first;
+      long long i = 0;
+      int stage = 0;
+      uint32_t round = 0;
+      bool dead = false;
+      int s = 0, k = 0, b = 0;
+      const int32_t* ptab = nullptr;
+      int cur = -1;
+      for (long long g = g_begin; g < g_end; ++g, ++i) {
+        while (pre[u + 1] <= g) ++u;
+        if (u != cur) {
+          cur = u;
+          s = u % p.kvp;
+          const int bk = u / p.kvp;
+          k = bk % p.Hkv;
+          b = bk / p.Hkv;
+          ptab = p.page_table + ((size_t)s * p.B + b) * p.max_pages;
+        }
+        const int pg = (int)(g - pre[u]);
+        if (*(volatile int*)&tail->abort_) { dead = true; break; }
+        if (round > 0 && !mbar_wait(&tail->empty[stage], (round - 1) & 1)) {
+          raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
+          *(volatile int*)&tail->abort_ = 1;
+          dead = true;
+          break;
+        }
+        const int page = __ldg(ptab + pg);
+        if (page < 0 || page >= p.num_pages) {
+          raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
+          mbar_arrive(&tail->full[stage]);  // completes the phase with no data; consumers skip
+        } else {
+          uint8_t* st = stages + (size_t)stage * Cfg::STAGE_BYTES;
+          const int row = (page * p.Hkv + k) * kPage;
+          mbar_arrive_expect_tx(&tail->full[stage], Cfg::STAGE_BYTES);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            tma_load_2d(st + c * kChunkBytes, &tmK, c * 64, row, &tail->full[stage]);
+            tma_load_2d(st + (NCH + c) * kChunkBytes, &tmV, c * 64, row, &tail->full[stage]);
+          }
+        }
+        if (++stage == NSTAGE) { stage = 0; ++round; }
+      }
+      if (dead) {  // let every load already issued land before the CTA exits
+        const long long n_issued = i;
+        for (long long j = n_issued > NSTAGE ? n_issued - NSTAGE : 0; j < n_issued; ++j)
+          mbar_wait(&tail->full[j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
+      }
+    }
+    return;
+  }
+
+  // ======================================= consumers ============================================
+  const int grp = warp / 4;   // which warpgroup: takes pages i with i % 2 == grp
+  const int w4 = warp & 3;    // token slice [16 w4, 16 w4 + 16) of the page
+  const int g8 = lane >> 2;   // fragment row (query head) g and g + 8
+  const int t4 = lane & 3;
+  const int tok0 = 16 * w4;
+  const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: which 8x8 matrix this lane addresses
+
+  uint32_t qa[KSTEPS][4];
+  float O[NT][4];
+  float m_run[2], l_run[2];
+  auto reset_state = [&]() {
+#pragma unroll
+    for (int j = 0; j < NT; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+  };
+  auto load_q = [&](int u) {
+    const int bk = u / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
+    const __nv_bfloat16* qb = p.q + ((size_t)b * p.Hq + (size_t)k * p.G) * D;
+    const bool v0 = g8 < p.G, v1 = g8 + 8 < p.G;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      const int c0 = 16 * kk + 2 * t4;
+      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qb + (size_t)g8 * D);
+      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qb + (size_t)(g8 + 8) * D);
+      qa[kk][0] = v0 ? __ldg(r0 + c0 / 2) : 0u;
+      qa[kk][1] = v1 ? __ldg(r1 + c0 / 2) : 0u;
+      qa[kk][2] = v0 ? __ldg(r0 + (c0 + 8) / 2) : 0u;
+      qa[kk][3] = v1 ? __ldg(r1 + (c0 + 8) / 2) : 0u;
+    }
+  };
+
+  reset_state();
+  int u = u_first;
+  int s_u = 0, b_u = 0, k_u = 0, len_u = 0;
+  const int32_t* ptab = nullptr;
+  auto enter_unit = [&](int uu) {
+    s_u = uu % p.kvp;
+    const int bk = uu / p.kvp;
+    k_u = bk % p.Hkv;
+    b_u = bk / p.Hkv;
+    len_u = p.shard_lens[s_u * p.B + b_u];
+    ptab = p.page_table + ((size_t)s_u * p.B + b_u) * p.max_pages;
+    load_q(uu);
+  };
+  enter_unit(u);
+  long long seg_begin = g_begin;
+  bool dead = false;
+  int stage = 0, parity = 0, gsel = 0;
+  const float sl2 = p.scale_log2;
+
+  for (long long g = g_begin; g < g_end; ++g) {
+    if (pre[u + 1] <= g) {  // entered a new unit
+      while (pre[u + 1] <= g) ++u;
+      enter_unit(u);
+    }
+    const int pg = (int)(g - pre[u]);
+    if (gsel == grp) {
+      if (!dead && *(volatile int*)&tail->abort_) dead = true;
+      if (!dead && !warp_wait(&tail->full[stage], parity)) {
+        if (lane == 0) {
+          raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
+          *(volatile int*)&tail->abort_ = 1;
+        }
+        dead = true;
+      }
+      if (!dead) {
+        const int page = __ldg(ptab + pg);
+        const int nvalid = min(kPage, len_u - pg * kPage);
+        uint8_t* st = stages + (size_t)stage * Cfg::STAGE_BYTES;
+        const bool page_ok = page >= 0 && page < p.num_pages;
+        if (page_ok && tok0 < nvalid) {
+          const uint32_t kbase = smem_u32(st);
+          const uint32_t vbase = kbase + NCH * kChunkBytes;
+          // zero the V rows past the end of the history in this warp's slice (0 * garbage = NaN)
+          if (tok0 + 16 > nvalid) {
+            for (int e = lane; e < 16 * NCH * 8; e += 32) {
+              const int row = tok0 + e / (NCH * 8);
+              const int rem = e % (NCH * 8);
+              if (row >= nvalid)
+                *reinterpret_cast<uint4*>(st + (NCH + rem / 8) * kChunkBytes + row * 128 +
+                                          (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+          // S = q K^T over this warp's 16 tokens: two n-tiles of 8 tokens
+          float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+          {
+            const int token = tok0 + (mi >> 1) * 8 + r8;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+              const int dch = 2 * kk + (mi & 1);  // 16-byte column chunk of the row
+              const uint32_t addr = kbase + (dch >> 3) * kChunkBytes + token * 128 +
+                                    ((((dch & 7) ^ (token & 7))) << 4);
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4(addr, b0, b1, b2, b3);
+              mma_bf16_16816(s0, qa[kk], b0, b1);
+              mma_bf16_16816(s1, qa[kk], b2, b3);
+            }
+          }
+          // online softmax (base 2)
+          const int ta = tok0 + 2 * t4, tb = tok0 + 8 + 2 * t4;
+          float x[8];
+          x[0] = ta < nvalid ? s0[0] * sl2 : -INFINITY;
+          x[1] = ta + 1 < nvalid ? s0[1] * sl2 : -INFINITY;
+          x[2] = tb < nvalid ? s1[0] * sl2 : -INFINITY;
+          x[3] = tb + 1 < nvalid ? s1[1] * sl2 : -INFINITY;
+          x[4] = ta < nvalid ? s0[2] * sl2 : -INFINITY;
+          x[5] = ta + 1 < nvalid ? s0[3] * sl2 : -INFINITY;
+          x[6] = tb < nvalid ? s1[2] * sl2 : -INFINITY;
+          x[7] = tb + 1 < nvalid ? s1[3] * sl2 : -INFINITY;
+          float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+          float mx1 = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+          const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+          const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+          const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+          const float al0 = fast_exp2(m_run[0] - mu0), al1 = fast_exp2(m_run[1] - mu1);
+          m_run[0] = mn0;
+          m_run[1] = mn1;
+          uint32_t pa[4];
+          pa[0] = pack_bf16x2(fast_exp2(x[0] - mu0), fast_exp2(x[1] - mu0));  // row g,   k 2t..
+          pa[1] = pack_bf16x2(fast_exp2(x[4] - mu1), fast_exp2(x[5] - mu1));  // row g+8, k 2t..
+          pa[2] = pack_bf16x2(fast_exp2(x[2] - mu0), fast_exp2(x[3] - mu0));  // row g,   k 8+2t..
+          pa[3] = pack_bf16x2(fast_exp2(x[6] - mu1), fast_exp2(x[7] - mu1));  // row g+8, k 8+2t..
+          // the row sums use the same bf16-rounded weights the tensor cores multiply by
+          l_run[0] = l_run[0] * al0 + (bf16_lo_to_f32(pa[0]) + bf16_hi_to_f32(pa[0])) +
+                     (bf16_lo_to_f32(pa[2]) + bf16_hi_to_f32(pa[2]));
+          l_run[1] = l_run[1] * al1 + (bf16_lo_to_f32(pa[1]) + bf16_hi_to_f32(pa[1])) +
+                     (bf16_lo_to_f32(pa[3]) + bf16_hi_to_f32(pa[3]));
+          if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+              O[j][0] *= al0;
+              O[j][1] *= al0;
+              O[j][2] *= al1;
+              O[j][3] *= al1;
+            }
+          }
+          // O += P V over the 16 tokens: V^T fragments via transposing ldmatrix
+          {
+            const int token = tok0 + (mi & 1) * 8 + r8;
+#pragma unroll
+            for (int n2 = 0; n2 < NT / 2; ++n2) {
+              const int dch = 2 * n2 + (mi >> 1);
+              const uint32_t addr = vbase + (dch >> 3) * kChunkBytes + token * 128 +
+                                    ((((dch & 7) ^ (token & 7))) << 4);
+              uint32_t v0, v1, v2, v3;
+              ldsm_x4_trans(addr, v0, v1, v2, v3);
+              mma_bf16_16816(O[2 * n2], pa, v0, v1);
+              mma_bf16_16816(O[2 * n2 + 1], pa, v2, v3);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tail->empty[stage]);
+      }
+    }
+    if (++gsel == kGroups) gsel = 0;
+    if (++stage == NSTAGE) { stage = 0; parity ^= 1; }
+
+    // ---- end of a segment: the unit ends here or the CTA's range does ----
+    if (g + 1 == g_end || g + 1 == pre[u + 1]) {
+      const int cw = warp;  // consumer warp 0..7
+      float l0 = l_run[0], l1 = l_run[1];
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      if (t4 == 0) {
+        tail->mstat[cw][g8] = m_run[0];
+        tail->mstat[cw][g8 + 8] = m_run[1];
+        tail->lstat[cw][g8] = l0;
+        tail->lstat[cw][g8 + 8] = l1;
+      }
+      named_barrier_sync(1, kConsumerWarps * 32);
+      {
+        float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          M0 = fmaxf(M0, tail->mstat[w][g8]);
+          M1 = fmaxf(M1, tail->mstat[w][g8 + 8]);
+        }
+        const float a0 = fast_exp2(m_run[0] - (M0 == -INFINITY ? 0.f : M0));
+        const float a1 = fast_exp2(m_run[1] - (M1 == -INFINITY ? 0.f : M1));
+        if (l0 > 0.f || l1 > 0.f) {
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            float* r0 = Obuf + g8 * D + 8 * j + 2 * t4;
+            float* r1 = r0 + 8 * D;
+            atomicAdd(r0, O[j][0] * a0);
+            atomicAdd(r0 + 1, O[j][1] * a0);
+            atomicAdd(r1, O[j][2] * a1);
+            atomicAdd(r1 + 1, O[j][3] * a1);
+          }
+        }
+      }
+      named_barrier_sync(1, kConsumerWarps * 32);
+
+      // every consumer thread owns row r, columns [c0, c0 + D/16)
+      const int r = tid / 16;
+      const int c0 = (tid % 16) * (D / 16);
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, tail->mstat[w][r]);
+      const float Mu = M == -INFINITY ? 0.f : M;
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w)
+        L += tail->lstat[w][r] * fast_exp2(tail->mstat[w][r] - Mu);
+
+      const size_t orow = ((size_t)s_u * p.B + b_u) * p.Hq + (size_t)k_u * p.G + r;
+      const bool whole = seg_begin == pre[u] && g + 1 == pre[u + 1];
+      if (whole) {
+        if (r < p.G) {
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          float* dst = p.o_part + orow * D + c0;
+#pragma unroll
+          for (int c = 0; c < D / 16; c += 4)
+            *reinterpret_cast<float4*>(dst + c) =
+                make_float4(Obuf[r * D + c0 + c] * inv, Obuf[r * D + c0 + c + 1] * inv,
+                            Obuf[r * D + c0 + c + 2] * inv, Obuf[r * D + c0 + c + 3] * inv);
+          if (c0 == 0) p.lse[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) Obuf[r * D + c0 + c] = 0.f;
+      } else {
+        const int slot = (g_begin >= pre[u]) ? 0 : 1;
+        float* rec = p.seg + ((size_t)blockIdx.x * 2 + slot) * GqaCfg<D>::REC;
+#pragma unroll
+        for (int c = 0; c < D / 16; c += 4) {
+          *reinterpret_cast<float4*>(rec + r * D + c0 + c) =
+              make_float4(Obuf[r * D + c0 + c], Obuf[r * D + c0 + c + 1],
+                          Obuf[r * D + c0 + c + 2], Obuf[r * D + c0 + c + 3]);
+        }
+        if (c0 == 0) {
+          rec[kRows * D + r] = M;
+          rec[kRows * D + kRows + r] = L;
+        }
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) Obuf[r * D + c0 + c] = 0.f;
+        __threadfence();
+        named_barrier_sync(1, kConsumerWarps * 32);
+        const int c_lo = cta_of(pre[u], W, Geff);
+        const int c_hi = cta_of((long long)pre[u + 1] - 1, W, Geff);
+        if (tid == 0) {
+          const int ticket = atomicAdd(&p.tickets[u], 1);
+          tail->flag = (ticket == c_hi - c_lo) ? 1 : 0;
+        }
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (tail->flag) {  // last arriver merges every segment of this unit
+          __threadfence();
+          float Mm = -INFINITY;
+          for (int c = c_lo; c <= c_hi; ++c) {
+            const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
+            const float* rc = p.seg + ((size_t)c * 2 + sl) * GqaCfg<D>::REC;
+            Mm = fmaxf(Mm, __ldcg(rc + kRows * D + r));
+          }
+          const float Mmu = Mm == -INFINITY ? 0.f : Mm;
+          float acc[D / 16];
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) acc[c] = 0.f;
+          float Lm = 0.f;
+          for (int c = c_lo; c <= c_hi; ++c) {
+            const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
+            const float* rc = p.seg + ((size_t)c * 2 + sl) * GqaCfg<D>::REC;
+            const float wgt = fast_exp2(__ldcg(rc + kRows * D + r) - Mmu);
+            Lm += __ldcg(rc + kRows * D + kRows + r) * wgt;
+#pragma unroll
+            for (int cc = 0; cc < D / 16; cc += 4) {
+              const float4 v = __ldcg(reinterpret_cast<const float4*>(rc + r * D + c0 + cc));
+              acc[cc] += v.x * wgt;
+              acc[cc + 1] += v.y * wgt;
+              acc[cc + 2] += v.z * wgt;
+              acc[cc + 3] += v.w * wgt;
+            }
+          }
+          if (r < p.G) {
+            const float inv = Lm > 0.f ? 1.f / Lm : 0.f;
+            float* dst = p.o_part + orow * D + c0;
+#pragma unroll
+            for (int c = 0; c < D / 16; c += 4)
+              *reinterpret_cast<float4*>(dst + c) =
+                  make_float4(acc[c] * inv, acc[c + 1] * inv, acc[c + 2] * inv, acc[c + 3] * inv);
+            if (c0 == 0) p.lse[orow] = Lm > 0.f ? (Mm + log2f(Lm)) * kLn2 : -INFINITY;
+          }
+          if (tid == 0) p.tickets[u] = 0;  // ready for the next launch
+        }
+      }
+      named_barrier_sync(1, kConsumerWarps * 32);
+      reset_state();
+      seg_begin = g + 1;
+    }
+  }
+}
+
+}  // namespace
+
+template <int D>
+static helix_status launch_bf16(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                const GqaParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = smem_bytes_for<D>(p.units);
+  auto kern = gqa_partial_bf16_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return HELIX_ERR_CUDA;
+  kern<<<grid, kThreads, smem, stream>>>(tmK, tmV, p);
+  return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
+}
+
+size_t gqa_partial_smem_bytes(int head_dim, int units) {
+  return head_dim == 64 ? smem_bytes_for<64>(units) : smem_bytes_for<128>(units);
+}
+
+size_t gqa_segment_record_floats(int head_dim) {
+  return head_dim == 64 ? GqaCfg<64>::REC : GqaCfg<128>::REC;
+}
+
+helix_status gqa_partial_bf16_launch(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                     const GqaParams& p, int grid, cudaStream_t stream) {
+  if (p.D == 128) return launch_bf16<128>(tmK, tmV, p, grid, stream);
+  if (p.D == 64) return launch_bf16<64>(tmK, tmV, p, grid, stream);
+  return HELIX_ERR_UNSUPPORTED;
+}
+
+}  // namespace helix

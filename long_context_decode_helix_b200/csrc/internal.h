@@ -1,0 +1,55 @@
+// internal.h -- host-side declarations shared by the helix translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "helix.h"
+
+namespace helix {
+
+// Parameters of the GQA partial kernels (bf16 and NVFP4 KV).
+struct GqaParams {
+  const __nv_bfloat16* q;     // [B][Hq][D]
+  const int32_t* page_table;  // [kvp][B][max_pages]
+  const int32_t* shard_lens;  // [kvp][B]
+  float* o_part;              // [kvp][B][Hq][D]
+  float* lse;                 // [kvp][B][Hq]
+  int32_t* tickets;           // [units], zero between launches
+  float* seg;                 // [grid][2][record]
+  uint32_t* err;              // may be null
+  const uint8_t* k_scale;     // NVFP4 only: [pages][Hkv][64][D/16]
+  const uint8_t* v_scale;
+  const uint8_t* k_codes;     // NVFP4 only: [pages][Hkv][64][D/2]
+  const uint8_t* v_codes;
+  int B, Hq, Hkv, G, D, kvp, max_pages, num_pages, units;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+size_t gqa_partial_smem_bytes(int head_dim, int units);
+size_t gqa_segment_record_floats(int head_dim);
+helix_status gqa_partial_bf16_launch(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                     const GqaParams& p, int grid, cudaStream_t stream);
+
+// Append: copies the new tokens' rows (and scales) into their pages.
+struct AppendParams {
+  const uint8_t* src[4];   // k rows, v rows, k scales, v scales (null when unused)
+  uint8_t* dst[4];         // matching pools
+  int row_bytes[4];        // bytes per (token, head) row of each stream; 0 = unused
+  const int32_t* page_table;
+  int32_t* shard_lens;
+  int32_t* seq_lens;
+  uint32_t* err;
+  const int32_t* n_valid;  // optional [B]
+  int B, Hkv, kvp, layout, rr_block, contig_chunk, page_tokens, max_pages, num_pages, n_new;
+};
+helix_status append_launch(const AppendParams& p, cudaStream_t stream);
+
+helix_status combine_launch(int kvp, int batch, int num_q_heads, int v_dim, const float* o_partial,
+                            const float* lse, void* o_out, int o_dtype, float* lse_out,
+                            cudaStream_t stream);
+
+}  // namespace helix

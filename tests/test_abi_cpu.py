@@ -1,0 +1,89 @@
+"""The C-ABI library loads on a CPU-only host, exports every declared symbol, and its host-side
+validation rejects bad arguments before touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(helix_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def hx():
+    import long_context_decode_helix_b200 as m
+
+    return m
+
+
+def test_every_declared_symbol_is_exported(hx):
+    names = _declared()
+    assert {"helix_kv_append", "helix_attn_partial", "helix_attn_combine"} <= set(names)
+    for n in names:
+        assert hasattr(hx.lib, n), f"libhelix.so does not export {n}"
+
+
+def test_status_strings(hx):
+    for code, name in hx.STATUS_NAMES.items():
+        assert hx.lib.helix_status_string(code).decode() == name
+    assert hx.lib.helix_version() >= 100
+
+
+def test_combine_rejects_bad_arguments(hx):
+    f = hx.lib.helix_attn_combine
+    buf = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    assert f(0, 1, 1, 4, buf, buf, buf, 0, None, None) == 1  # kvp = 0
+    assert f(1, 1, 1, 6, buf, buf, buf, 0, None, None) == 1  # v_dim not a multiple of 4
+    assert f(1, 1, 1, 4, None, buf, buf, 0, None, None) == 1  # null o_partial
+    assert f(1, 1, 1, 4, buf, buf, buf, 7, None, None) == 1  # bad o_dtype
+    assert f(1, 1, 1, 4, ctypes.c_void_p(8), buf, buf, 0, None, None) == 1  # misaligned
+
+
+def _struct(hx, **kw):
+    base = dict(kind=0, kv_dtype=0, layout=0, kvp=8, batch=8, num_kv_heads=8, head_dim=128,
+                v_dim=128, page_tokens=64, rr_block=16, contig_chunk=0, num_pages=16,
+                max_pages_per_shard=2, reserved_=0, k_pool=4096, v_pool=8192, k_scale=None,
+                v_scale=None, page_table=256, shard_lens=512, seq_lens=768, err_word=None)
+    base.update(kw)
+    return hx.CacheStruct(**base)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(kvp=0), dict(batch=0), dict(num_kv_heads=0), dict(layout=5), dict(kind=9),
+    dict(rr_block=0), dict(layout=1, contig_chunk=0), dict(k_pool=None), dict(v_pool=None),
+    dict(k_pool=4100), dict(page_table=None), dict(seq_lens=None), dict(v_dim=64),
+    dict(kv_dtype=1), dict(kind=1, num_kv_heads=1, head_dim=576, v_dim=512),  # MLA needs v_pool NULL
+])
+def test_append_rejects_bad_cache(hx, bad):
+    s = _struct(hx, **bad)
+    k = ctypes.c_void_p(1 << 20)
+    assert hx.lib.helix_kv_append(ctypes.byref(s), k, k, None, None, 1, None, None) == 1
+
+
+def test_append_capacity_check(hx):
+    s = _struct(hx, num_pages=1 << 24, num_kv_heads=64, page_tokens=64, batch=1, kvp=1)
+    k = ctypes.c_void_p(1 << 20)
+    assert hx.lib.helix_kv_append(ctypes.byref(s), k, k, None, None, 1, None, None) == 3
+
+
+def test_null_cache_and_negative_n(hx):
+    assert hx.lib.helix_kv_append(None, None, None, None, None, 1, None, None) == 1
+    s = _struct(hx)
+    k = ctypes.c_void_p(1 << 20)
+    assert hx.lib.helix_kv_append(ctypes.byref(s), k, k, None, None, -1, None, None) == 1
+    assert hx.lib.helix_kv_append(ctypes.byref(s), k, k, None, None, 0, None, None) == 0  # no-op
+    n = ctypes.c_size_t()
+    assert hx.lib.helix_attn_workspace_size(None, 128, ctypes.byref(n)) == 1
+    assert hx.lib.helix_attn_workspace_size(ctypes.byref(s), 100, ctypes.byref(n)) == 1  # Hq % Hkv
+    assert hx.lib.helix_attn_workspace_size(ctypes.byref(s), 256, ctypes.byref(n)) == 2  # G = 32

@@ -184,6 +184,29 @@ def kv_range_nvfp4(w, which, b, h, t0, t1, device="cpu"):
     return nvfp4_encode(kv_range_f32(w, which, b, h, t0, t1, device))
 
 
+def append_rows(w: Workload, t0: int, t1: int, device="cpu") -> dict:
+    """The arguments of one append call for history positions [t0, t1) of every request:
+    bf16 k_new/v_new [B, n, Hkv, d] (GQA), NVFP4 codes and scales (GQA NVFP4) or the latent rows
+    k_new [B, n, d] (MLA)."""
+    if w.kind == "mla":
+        c = torch.stack([kv_range_bf16(w, "c", b, 0, t0, t1, device) for b in range(w.B)])
+        return dict(k_new=c.contiguous())
+    if w.kv_dtype == "nvfp4":
+        out = {}
+        for which in ("k", "v"):
+            codes = [[None] * w.Hkv for _ in range(w.B)]
+            scales = [[None] * w.Hkv for _ in range(w.B)]
+            for b in range(w.B):
+                for h in range(w.Hkv):
+                    codes[b][h], scales[b][h] = kv_range_nvfp4(w, which, b, h, t0, t1, device)
+            out[which + "_new"] = torch.stack([torch.stack(c, 1) for c in codes]).contiguous()
+            out[which + "_scale"] = torch.stack([torch.stack(c, 1) for c in scales]).contiguous()
+        return out
+    k = torch.stack([kv_tokens(w, "k", b, t0, t1, device) for b in range(w.B)]).contiguous()
+    v = torch.stack([kv_tokens(w, "v", b, t0, t1, device) for b in range(w.B)]).contiguous()
+    return dict(k_new=k, v_new=v)
+
+
 # ----------------------------------------------------------------------------------------------
 # paging
 
