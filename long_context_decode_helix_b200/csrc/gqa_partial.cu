@@ -42,7 +42,8 @@ struct GqaCfg {
   static constexpr int NCH = D / 64;                        // 64-column halves per row
   static constexpr int STAGE_BYTES = 2 * NCH * kChunkBytes;  // K + V of one (page, kv head)
   static constexpr int NSTAGE = (D == 128) ? 5 : 10;
-  static constexpr int REC = kRows * (D + 2);  // floats per workspace segment record
+  // floats per workspace segment record: O [16][D], then m, l, lb per row
+  static constexpr int REC = kRows * (D + 3);
 };
 
 struct SmemTail {
@@ -50,6 +51,7 @@ struct SmemTail {
   uint64_t empty[16];
   float mstat[kConsumerWarps][kRows];
   float lstat[kConsumerWarps][kRows];
+  float lbstat[kConsumerWarps][kRows];
   int flag;
   int abort_;
 };
@@ -57,7 +59,8 @@ struct SmemTail {
 template <int D>
 __host__ __device__ constexpr size_t smem_bytes_for(int units) {
   return 1024 /*alignment slack*/ + (size_t)GqaCfg<D>::NSTAGE * GqaCfg<D>::STAGE_BYTES +
-         (size_t)kRows * D * sizeof(float) + sizeof(SmemTail) + (size_t)(units + 1) * sizeof(int);
+         4 * (size_t)kRows * D * sizeof(float) + sizeof(SmemTail) +
+         (size_t)(units + 1) * sizeof(int);
 }
 
 __device__ __forceinline__ long long range_begin(int c, long long W, int G) {
@@ -90,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* stages = smem;
   float* Obuf = reinterpret_cast<float*>(smem + (size_t)NSTAGE * Cfg::STAGE_BYTES);
-  SmemTail* tail = reinterpret_cast<SmemTail*>(Obuf + kRows * D);
+  SmemTail* tail = reinterpret_cast<SmemTail*>(Obuf + 4 * kRows * D);
   int* pre = reinterpret_cast<int*>(tail + 1);
 
   const int tid = threadIdx.x;
@@ -110,7 +113,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     pre[u + 1] = np;
   }
-  for (int i = tid; i < kRows * D; i += kThreads) Obuf[i] = 0.f;
   if (tid == 0) {
     pre[0] = 0;
     tail->flag = 0;
@@ -232,12 +234,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t qa[KSTEPS][4];
   float O[NT][4];
-  float m_run[2], l_run[2];
+  // m: running max (base-2 logits); l: sum of fp32 weights (for the LSE); lb: sum of the
+  // bf16-rounded weights the tensor cores multiply V by (normalises O, so O stays a convex
+  // combination of V rows to fp32 accuracy)
+  float m_run[2], l_run[2], lb_run[2];
   auto reset_state = [&]() {
 #pragma unroll
     for (int j = 0; j < NT; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
     m_run[0] = m_run[1] = -INFINITY;
     l_run[0] = l_run[1] = 0.f;
+    lb_run[0] = lb_run[1] = 0.f;
   };
   auto load_q = [&](int u) {
     const int bk = u / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
@@ -347,16 +353,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float al0 = fast_exp2(m_run[0] - mu0), al1 = fast_exp2(m_run[1] - mu1);
           m_run[0] = mn0;
           m_run[1] = mn1;
+          float pw[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pw[e] = fast_exp2(x[e] - mu0);
+#pragma unroll
+          for (int e = 4; e < 8; ++e) pw[e] = fast_exp2(x[e] - mu1);
           uint32_t pa[4];
-          pa[0] = pack_bf16x2(fast_exp2(x[0] - mu0), fast_exp2(x[1] - mu0));  // row g,   k 2t..
-          pa[1] = pack_bf16x2(fast_exp2(x[4] - mu1), fast_exp2(x[5] - mu1));  // row g+8, k 2t..
-          pa[2] = pack_bf16x2(fast_exp2(x[2] - mu0), fast_exp2(x[3] - mu0));  // row g,   k 8+2t..
-          pa[3] = pack_bf16x2(fast_exp2(x[6] - mu1), fast_exp2(x[7] - mu1));  // row g+8, k 8+2t..
-          // the row sums use the same bf16-rounded weights the tensor cores multiply by
-          l_run[0] = l_run[0] * al0 + (bf16_lo_to_f32(pa[0]) + bf16_hi_to_f32(pa[0])) +
-                     (bf16_lo_to_f32(pa[2]) + bf16_hi_to_f32(pa[2]));
-          l_run[1] = l_run[1] * al1 + (bf16_lo_to_f32(pa[1]) + bf16_hi_to_f32(pa[1])) +
-                     (bf16_lo_to_f32(pa[3]) + bf16_hi_to_f32(pa[3]));
+          pa[0] = pack_bf16x2(pw[0], pw[1]);  // row g,   k 2t..
+          pa[1] = pack_bf16x2(pw[4], pw[5]);  // row g+8, k 2t..
+          pa[2] = pack_bf16x2(pw[2], pw[3]);  // row g,   k 8+2t..
+          pa[3] = pack_bf16x2(pw[6], pw[7]);  // row g+8, k 8+2t..
+          l_run[0] = l_run[0] * al0 + ((pw[0] + pw[1]) + (pw[2] + pw[3]));
+          l_run[1] = l_run[1] * al1 + ((pw[4] + pw[5]) + (pw[6] + pw[7]));
+          lb_run[0] = lb_run[0] * al0 + (bf16_lo_to_f32(pa[0]) + bf16_hi_to_f32(pa[0])) +
+                      (bf16_lo_to_f32(pa[2]) + bf16_hi_to_f32(pa[2]));
+          lb_run[1] = lb_run[1] * al1 + (bf16_lo_to_f32(pa[1]) + bf16_hi_to_f32(pa[1])) +
+                      (bf16_lo_to_f32(pa[3]) + bf16_hi_to_f32(pa[3]));
           if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
@@ -396,11 +408,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      float lb0 = lb_run[0], lb1 = lb_run[1];
+      lb0 += __shfl_xor_sync(0xffffffffu, lb0, 1);
+      lb0 += __shfl_xor_sync(0xffffffffu, lb0, 2);
+      lb1 += __shfl_xor_sync(0xffffffffu, lb1, 1);
+      lb1 += __shfl_xor_sync(0xffffffffu, lb1, 2);
       if (t4 == 0) {
         tail->mstat[cw][g8] = m_run[0];
         tail->mstat[cw][g8 + 8] = m_run[1];
         tail->lstat[cw][g8] = l0;
         tail->lstat[cw][g8 + 8] = l1;
+        tail->lbstat[cw][g8] = lb0;
+        tail->lbstat[cw][g8 + 8] = lb1;
       }
       named_barrier_sync(1, kConsumerWarps * 32);
       {
@@ -412,15 +431,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float a0 = fast_exp2(m_run[0] - (M0 == -INFINITY ? 0.f : M0));
         const float a1 = fast_exp2(m_run[1] - (M1 == -INFINITY ? 0.f : M1));
-        if (l0 > 0.f || l1 > 0.f) {
 #pragma unroll
-          for (int j = 0; j < NT; ++j) {
+        for (int j = 0; j < NT; ++j) {
+          O[j][0] *= a0;
+          O[j][1] *= a0;
+          O[j][2] *= a1;
+          O[j][3] *= a1;
+        }
+      }
+      // Sum the 8 warps' O in a fixed order (4+4, 2+2, 1+1) so results are bit-reproducible.
+      // Four 16 x D buffers; every warp only overwrites a buffer it has finished reading itself.
+      {
+        auto put = [&](int slot) {
+          float* dst = Obuf + slot * kRows * D;
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[(j * 4 + e) * 32 + lane] = O[j][e];
+        };
+        auto add = [&](int slot) {
+          const float* src = Obuf + slot * kRows * D;
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) O[j][e] += src[(j * 4 + e) * 32 + lane];
+        };
+        if (cw >= 4) put(cw - 4);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (cw < 4) add(cw);
+        __syncwarp();
+        if (cw == 2 || cw == 3) put(cw);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (cw < 2) add(cw + 2);
+        __syncwarp();
+        if (cw == 1) put(1);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (cw == 0) {
+          add(1);
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {  // natural [row][column] layout for the output phase
             float* r0 = Obuf + g8 * D + 8 * j + 2 * t4;
-            float* r1 = r0 + 8 * D;
-            atomicAdd(r0, O[j][0] * a0);
-            atomicAdd(r0 + 1, O[j][1] * a0);
-            atomicAdd(r1, O[j][2] * a1);
-            atomicAdd(r1 + 1, O[j][3] * a1);
+            r0[0] = O[j][0];
+            r0[1] = O[j][1];
+            r0[8 * D] = O[j][2];
+            r0[8 * D + 1] = O[j][3];
           }
         }
       }
@@ -433,16 +488,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, tail->mstat[w][r]);
       const float Mu = M == -INFINITY ? 0.f : M;
-      float L = 0.f;
+      float L = 0.f, LB = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w)
-        L += tail->lstat[w][r] * fast_exp2(tail->mstat[w][r] - Mu);
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float e = fast_exp2(tail->mstat[w][r] - Mu);
+        L += tail->lstat[w][r] * e;
+        LB += tail->lbstat[w][r] * e;
+      }
 
       const size_t orow = ((size_t)s_u * p.B + b_u) * p.Hq + (size_t)k_u * p.G + r;
       const bool whole = seg_begin == pre[u] && g + 1 == pre[u + 1];
       if (whole) {
         if (r < p.G) {
-          const float inv = L > 0.f ? 1.f / L : 0.f;
+          const float inv = LB > 0.f ? 1.f / LB : 0.f;
           float* dst = p.o_part + orow * D + c0;
 #pragma unroll
           for (int c = 0; c < D / 16; c += 4)
@@ -451,8 +509,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             Obuf[r * D + c0 + c + 2] * inv, Obuf[r * D + c0 + c + 3] * inv);
           if (c0 == 0) p.lse[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
         }
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) Obuf[r * D + c0 + c] = 0.f;
       } else {
         const int slot = (g_begin >= pre[u]) ? 0 : 1;
         float* rec = p.seg + ((size_t)blockIdx.x * 2 + slot) * GqaCfg<D>::REC;
@@ -465,9 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c0 == 0) {
           rec[kRows * D + r] = M;
           rec[kRows * D + kRows + r] = L;
+          rec[kRows * D + 2 * kRows + r] = LB;
         }
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) Obuf[r * D + c0 + c] = 0.f;
         __threadfence();
         named_barrier_sync(1, kConsumerWarps * 32);
         const int c_lo = cta_of(pre[u], W, Geff);
@@ -489,12 +544,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           float acc[D / 16];
 #pragma unroll
           for (int c = 0; c < D / 16; ++c) acc[c] = 0.f;
-          float Lm = 0.f;
+          float Lm = 0.f, LBm = 0.f;
           for (int c = c_lo; c <= c_hi; ++c) {
             const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
             const float* rc = p.seg + ((size_t)c * 2 + sl) * GqaCfg<D>::REC;
             const float wgt = fast_exp2(__ldcg(rc + kRows * D + r) - Mmu);
             Lm += __ldcg(rc + kRows * D + kRows + r) * wgt;
+            LBm += __ldcg(rc + kRows * D + 2 * kRows + r) * wgt;
 #pragma unroll
             for (int cc = 0; cc < D / 16; cc += 4) {
               const float4 v = __ldcg(reinterpret_cast<const float4*>(rc + r * D + c0 + cc));
@@ -505,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (r < p.G) {
-            const float inv = Lm > 0.f ? 1.f / Lm : 0.f;
+            const float inv = LBm > 0.f ? 1.f / LBm : 0.f;
             float* dst = p.o_part + orow * D + c0;
 #pragma unroll
             for (int c = 0; c < D / 16; c += 4)

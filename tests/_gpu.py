@@ -90,6 +90,7 @@ def assert_close_lse(got, want, what):
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     both = np.isneginf(got) & np.isneginf(want)
-    err = np.where(both, 0.0, np.abs(got - want))
+    with np.errstate(invalid="ignore"):
+        err = np.where(both, 0.0, np.abs(got - want))
     assert np.all(np.isfinite(err)), f"{what}: -inf mismatch"
     assert err.max(initial=0) <= TOL_LSE, f"{what}: max-abs {err.max():.3e} > {TOL_LSE}"
