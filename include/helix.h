@@ -158,6 +158,28 @@ helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads,
                                 const float* o_partial, const float* lse, void* o_out,
                                 int32_t o_dtype, float* lse_out, helix_stream_t stream);
 
+/*
+ * helix_attn_partial for callers that cannot allocate device memory. The paper has no counterpart;
+ * this is a deployment convenience of this library.
+ *
+ * Same arguments and results as helix_attn_partial, minus the workspace: the kernel's scratch lives
+ * in a fixed device array of HELIX_NOALLOC_SCRATCH_BYTES inside the library (one per GPU, held
+ * until the process exits). Meant for code that has no way to obtain a scratch buffer -- a plugin
+ * whose host owns all device memory, a fixed pre-reserved memory budget, or a loop that must never
+ * call cudaMalloc. The call allocates nothing.
+ *   - Returns HELIX_ERR_CAPACITY, launching nothing, when this cache shape needs more scratch than
+ *     HELIX_NOALLOC_SCRATCH_BYTES (see helix_attn_workspace_size).
+ *   - The first call on each device looks up the array's device address (once, with that device
+ *     current); make that first call before any stream capture.
+ *   - Each call zeroes the scratch it uses (an async memset on `stream`) before the kernel runs.
+ *   - All calls on one device share the array: calls that may run concurrently on the GPU race and
+ *     must be ordered by the caller (one stream, or events).
+ */
+#define HELIX_NOALLOC_SCRATCH_BYTES (4u << 20)
+helix_status helix_attn_partial_noalloc(const helix_kv_cache* cache, const void* q,
+                                        int32_t num_q_heads, float softmax_scale,
+                                        float* o_partial, float* lse, helix_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char* helix_status_string(helix_status status);
 

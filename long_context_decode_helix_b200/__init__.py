@@ -60,6 +60,8 @@ def _load():
     lib.helix_attn_workspace_size.restype = I32
     lib.helix_attn_partial.argtypes = [cache_p, P, I32, F32, P, P, P, SZ, P]
     lib.helix_attn_partial.restype = I32
+    lib.helix_attn_partial_noalloc.argtypes = [cache_p, P, I32, F32, P, P, P]
+    lib.helix_attn_partial_noalloc.restype = I32
     lib.helix_attn_combine.argtypes = [I32, I32, I32, I32, P, P, P, I32, P, P]
     lib.helix_attn_combine.restype = I32
     lib.helix_status_string.argtypes = [I32]
