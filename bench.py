@@ -38,7 +38,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="helix", choices=["helix", "reference"])
     ap.add_argument("--workload", default="gqa_s1m", choices=sorted(wl.WORKLOADS))
@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--cpu-sample-tokens", type=int, default=1 << 19,
                     help="history tokens per sampled head group for the CPU oracle")
     ap.add_argument("--cpu-sample-groups", type=int, default=4)
+    ap.add_argument("--context", type=int, default=None,
+                    help="override the history length (fixed lengths), e.g. for small profiling runs")
     return ap.parse_args()
 
 
@@ -152,14 +154,21 @@ def measured_peaks():
 
 
 def profile_traffic(kernel: str, workload: str):
-    """dram read+write bytes per launch from a committed ncu summary, when one exists for exactly
-    this kernel build; otherwise None."""
+    """dram read+write bytes per launch from a committed ncu summary, when one exists for this
+    workload and the kernel source is unchanged since the counters were taken; otherwise None."""
+    import hashlib
+
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    e = d.get(f"{kernel}:{workload}")
-    return None if e is None else e.get("dram_bytes_per_launch")
+    e = json.load(open(p)).get(f"{kernel}:{workload}")
+    if e is None:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return e["dram_bytes_per_launch"] if sha == e["source_sha256_16"] else None
 
 
 # ------------------------------------------------------------------------------------------------
@@ -249,6 +258,8 @@ def run_helix(args):
     import long_context_decode_helix_b200 as hx
 
     w = wl.WORKLOADS[args.workload]
+    if args.context is not None:
+        w = w.with_(S=args.context, S_min=None)
     lens = wl.seq_lens(w)
     dev = torch.device("cuda", local)
     K, W = args.steps, args.warmup
@@ -307,10 +318,12 @@ def run_helix(args):
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
+    torch.cuda.nvtx.range_push("timed_steps")
     start.record(stream)
     for i in range(K):
         one_step(si + i, evs[i])
     stop.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
