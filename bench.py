@@ -372,7 +372,8 @@ def run_helix(args):
         achieved_gbs = part_bytes / (part_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
                 "frac": achieved_gbs / peak, "peak_source": peak_kind,
-                "kernel": "gqa_partial_bf16_kernel" if w.kind == "gqa" else "mla_partial",
+                "kernel": ("mla_partial_kernel" if w.kind == "mla" else
+                           f"gqa_partial_kernel<{w.d},{w.kv_dtype}>"),
                 "bytes_per_launch": part_bytes,
                 "traffic": profile_traffic("partial", w.name)}
         line = {

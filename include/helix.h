@@ -72,8 +72,16 @@ typedef enum { HELIX_LAYOUT_RR = 0, HELIX_LAYOUT_CONTIG = 1 } helix_layout;
  *
  * Pool layouts (P = num_pages, H = num_kv_heads, T = page_tokens, d = head_dim):
  *   GQA, BF16 : k_pool, v_pool  bf16  [P][H][T][d]
- *   GQA, NVFP4: k_pool, v_pool  uint8 [P][H][T][d/2]   E2M1 codes, element 2i in the low nibble
- *               k_scale, v_scale uint8 [P][H][T][d/16] E4M3 scale of elements 16j..16j+15
+ *   GQA, NVFP4: k_pool  uint8 [P][H][T][d/2]  E2M1 codes of K, element 2i in the low nibble
+ *               k_scale uint8 [P][H][T][d/16] E4M3 scale of elements 16j..16j+15 of a K row
+ *               v_pool  uint8 [P][H][T/2][d]  E2M1 codes of V, token-pair interleaved: the byte
+ *                       for (pair i, column c) holds V[token 2i][c] in the low nibble and
+ *                       V[token 2i+1][c] in the high nibble (the P.V contraction runs over tokens,
+ *                       so its operands pair tokens); within pair row i it sits at byte
+ *                       16 * ((c / 16) XOR (2 * (i mod 4))) + c mod 16 (a bank-conflict swizzle)
+ *               v_scale uint8 [P][H][d/16][T] E4M3 scale of elements 16j..16j+15 of V row t, at [j][t]
+ *               helix_kv_append takes K and V rows in the same natural row format and does the
+ *               V re-layout.
  *   MLA, BF16 : k_pool          bf16  [P][T][d] with d = 576 (H = 1); V is columns [0, v_dim) of
  *               the same rows (v_pool must be NULL): keys and values share one latent row.
  *

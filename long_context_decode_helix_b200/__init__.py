@@ -126,11 +126,11 @@ class KVCache:
         t = self.tensors
         if self.kind == ATTN_MLA:
             t["k_pool"] = torch.zeros(P, T, d, dtype=torch.bfloat16, device=dev)
-        elif self.kv_dtype == KV_NVFP4:
-            for n in ("k_pool", "v_pool"):
-                t[n] = torch.zeros(P, H, T, d // 2, dtype=torch.uint8, device=dev)
-            for n in ("k_scale", "v_scale"):
-                t[n] = torch.zeros(P, H, T, d // 16, dtype=torch.uint8, device=dev)
+        elif self.kv_dtype == KV_NVFP4:  # V is stored token-pair interleaved (see helix.h)
+            t["k_pool"] = torch.zeros(P, H, T, d // 2, dtype=torch.uint8, device=dev)
+            t["k_scale"] = torch.zeros(P, H, T, d // 16, dtype=torch.uint8, device=dev)
+            t["v_pool"] = torch.zeros(P, H, T // 2, d, dtype=torch.uint8, device=dev)
+            t["v_scale"] = torch.zeros(P, H, d // 16, T, dtype=torch.uint8, device=dev)
         else:
             for n in ("k_pool", "v_pool"):
                 t[n] = torch.zeros(P, H, T, d, dtype=torch.bfloat16, device=dev)

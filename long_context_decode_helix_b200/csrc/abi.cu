@@ -85,7 +85,7 @@ helix_status check_cache(const helix_kv_cache* c) {
     if (c->v_pool == nullptr || !aligned16(c->v_pool)) return HELIX_ERR_INVALID_ARG;
     if (c->v_dim != c->head_dim) return HELIX_ERR_INVALID_ARG;
     if (c->kv_dtype == HELIX_KV_NVFP4) {
-      if (c->head_dim % 32 != 0) return HELIX_ERR_INVALID_ARG;
+      if (c->head_dim != 128) return HELIX_ERR_UNSUPPORTED;  // the V-code swizzle spans 8 chunks
       if (c->k_scale == nullptr || c->v_scale == nullptr || !aligned16(c->k_scale) ||
           !aligned16(c->v_scale))
         return HELIX_ERR_INVALID_ARG;
@@ -123,11 +123,12 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
   if (c->page_tokens != 64) return HELIX_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return HELIX_ERR_UNSUPPORTED;
   if (num_q_heads / c->num_kv_heads > 16) return HELIX_ERR_UNSUPPORTED;
-  if (c->kv_dtype != HELIX_KV_BF16) return HELIX_ERR_UNSUPPORTED;
+  const int nvfp4 = c->kv_dtype == HELIX_KV_NVFP4;
+  if (nvfp4 && c->head_dim != 128) return HELIX_ERR_UNSUPPORTED;
   int sms = 0, max_smem = 0;
   if (device_sm_count(&sms) != 0 || device_max_smem(&max_smem) != 0) return HELIX_ERR_CUDA;
   plan->units = c->batch * c->num_kv_heads * c->kvp;
-  if (gqa_partial_smem_bytes(c->head_dim, plan->units) > (size_t)max_smem)
+  if (gqa_partial_smem_bytes(c->head_dim, nvfp4, plan->units) > (size_t)max_smem)
     return HELIX_ERR_CAPACITY;
   plan->grid = sms;
   plan->ticket_bytes = (((size_t)plan->units * sizeof(int32_t)) + 255) & ~size_t(255);
@@ -178,6 +179,8 @@ helix_status helix_kv_append(const helix_kv_cache* c, const void* k_new, const v
     p.src[1] = (const uint8_t*)v_new; p.dst[1] = (uint8_t*)c->v_pool; p.row_bytes[1] = d / 2;
     p.src[2] = (const uint8_t*)k_new_scale; p.dst[2] = (uint8_t*)c->k_scale; p.row_bytes[2] = d / 16;
     p.src[3] = (const uint8_t*)v_new_scale; p.dst[3] = (uint8_t*)c->v_scale; p.row_bytes[3] = d / 16;
+    p.v_nvfp4 = 1;
+    if (c->page_tokens % 2 != 0 || d % 8 != 0) return HELIX_ERR_INVALID_ARG;
   } else {  // MLA: one latent row per token, V aliases its first v_dim columns
     if (k_new == nullptr || v_new != nullptr || !aligned4(k_new)) return HELIX_ERR_INVALID_ARG;
     p.src[0] = (const uint8_t*)k_new; p.dst[0] = (uint8_t*)c->k_pool; p.row_bytes[0] = d * 2;
@@ -243,6 +246,13 @@ helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t 
   p.num_pages = c->num_pages;
   p.units = plan.units;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (c->kv_dtype == HELIX_KV_NVFP4) {
+    p.k_codes = reinterpret_cast<const uint8_t*>(c->k_pool);
+    p.k_scale = reinterpret_cast<const uint8_t*>(c->k_scale);
+    p.v_codes = reinterpret_cast<const uint8_t*>(c->v_pool);
+    p.v_scale = reinterpret_cast<const uint8_t*>(c->v_scale);
+    return gqa_partial_nvfp4_launch(p, plan.grid, reinterpret_cast<cudaStream_t>(stream));
+  }
 
   const uint64_t rows = (uint64_t)c->num_pages * c->num_kv_heads * c->page_tokens;
   CUtensorMap tmK, tmV;

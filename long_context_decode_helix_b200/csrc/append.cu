@@ -119,11 +119,43 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
     }
     const size_t src_row = ((size_t)b * p.n_new + j) * p.Hkv + h;
     const size_t dst_row = ((size_t)page * p.Hkv + h) * p.page_tokens + slot;
+    if (!p.v_nvfp4) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int rb = p.row_bytes[k];
-      if (rb == 0) continue;
-      copy_bytes(p.dst[k] + dst_row * rb, p.src[k] + src_row * rb, rb, lane, 32);
+      for (int k = 0; k < 4; ++k) {
+        const int rb = p.row_bytes[k];
+        if (rb == 0) continue;
+        copy_bytes(p.dst[k] + dst_row * rb, p.src[k] + src_row * rb, rb, lane, 32);
+      }
+    } else {
+      // K codes and scales: natural rows
+      copy_bytes(p.dst[0] + dst_row * p.row_bytes[0], p.src[0] + src_row * p.row_bytes[0],
+                 p.row_bytes[0], lane, 32);
+      copy_bytes(p.dst[2] + dst_row * p.row_bytes[2], p.src[2] + src_row * p.row_bytes[2],
+                 p.row_bytes[2], lane, 32);
+      // V codes: element c of this token goes to nibble (slot & 1) of byte [slot / 2][c] of the
+      // (page, head) block, whose 16-byte chunks are XOR-swizzled by 2 (pair mod 4) (see helix.h).
+      // The other nibble belongs to the neighbouring token, which another warp (or another call)
+      // may be writing, so each 32-bit word is updated with atomic and/or.
+      const int d = p.row_bytes[1] * 2;
+      const int pair = slot / 2;
+      const uint8_t* vs = p.src[1] + src_row * p.row_bytes[1];
+      uint32_t* vblk = reinterpret_cast<uint32_t*>(
+          p.dst[1] + (((size_t)page * p.Hkv + h) * (p.page_tokens / 2) + pair) * d);
+      const int shift = 4 * (slot & 1);
+      for (int wd = lane; wd < d / 4; wd += 32) {  // word wd covers columns 4wd .. 4wd+3
+        const uint32_t two = *reinterpret_cast<const uint16_t*>(vs + 2 * wd);  // 4 codes
+        uint32_t bits = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) bits |= ((two >> (4 * e)) & 0xFu) << (8 * e + shift);
+        const int sw = ((((wd >> 2) ^ ((pair & 3) << 1))) << 2) | (wd & 3);
+        atomicAnd(vblk + sw, ~(0x0F0F0F0Fu << shift));
+        atomicOr(vblk + sw, bits);
+      }
+      // V scales: block-major, [block][token] inside the (page, head) block
+      const int nblk = p.row_bytes[3];
+      const uint8_t* ss = p.src[3] + src_row * nblk;
+      uint8_t* sblk = p.dst[3] + ((size_t)page * p.Hkv + h) * nblk * p.page_tokens;
+      for (int k = lane; k < nblk; k += 32) sblk[(size_t)k * p.page_tokens + slot] = ss[k];
     }
   }
   if (update_here) {

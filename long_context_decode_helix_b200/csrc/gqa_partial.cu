@@ -1,4 +1,4 @@
-// gqa_partial.cu -- per-shard partial decode attention for grouped-query attention, bf16 KV.
+// gqa_partial.cu -- per-shard partial decode attention for grouped-query attention (bf16 or NVFP4 KV).
 //
 // What it computes (paper summary "Helix Parallelism: Rethinking Sharding Strategies for
 // Interactive Multi-Million-Token LLM Decoding", fdeinterviews.com, paragraph on KV parallelism):
@@ -15,9 +15,25 @@
 // merged by whichever CTA arrives last on the unit's ticket (an atomic counter -- nobody spins).
 //
 // CTA layout: warps 0-7 are two consumer warpgroups that take alternate pages; warp w of a group owns
-// tokens [16w, 16w+16) of its page. Warp 8 is the producer: one lane issues TMA tile loads of the
-// page's K and V rows (128-byte swizzle, 8 KiB per 64-column half) into an NSTAGE-deep ring guarded by
-// mbarriers. Softmax is online in fp32 and base 2 (scale * log2 e folded into the logits).
+// tokens [16w, 16w+16) of its page. Warp 8 is the producer: it resolves the page ids of 32 pages at a
+// time with one coalesced load, and one lane issues the loads of each page into an NSTAGE-deep ring
+// guarded by mbarriers. NSTAGE is a multiple of the number of groups, so a stage is only ever used by
+// one group and no consumer can wait on a phase more than one ahead of the one it last consumed.
+// Softmax is online in fp32 and base 2 (scale * log2 e folded into the logits).
+//
+// bf16 KV: TMA tile loads of the page's K and V rows (128-byte swizzle, 8 KiB per 64-column half);
+// ldmatrix feeds the S = q K^T and P V tiles.
+//
+// NVFP4 KV (the pages' simulated results use FP4 KV: paper summary, roofline paragraph). The stage
+// is four 1-D bulk copies of one (page, KV head): K codes, K scales, V codes, V scales (9 KiB at
+// d = 128). E2M1 x E4M3 products are exact in f16 (at most 6 significant bits, 2^-10 .. 2688), so
+// each thread dequantises straight into f16 m16n8k16 fragments: one cvt.rn.f16x2.e2m1x2 and one
+// HMUL2 per two elements. For S = q K^T the MMA's k index is permuted so that a thread's 32
+// contiguous elements of a K row (one 16-byte load) are its B operands for all eight k-steps; q's
+// A fragments use the same permutation. For P V the pool stores V token-pair interleaved (see
+// helix.h), so a byte is already the (token 2i, token 2i+1) pair the B fragment needs, and V's n
+// index is permuted (output column 16 n + j for n-tile j) so one 16-byte load per token pair feeds
+// all sixteen n-tiles; the flush writes O back in natural column order.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,25 +46,36 @@
 namespace helix {
 namespace {
 
-constexpr int kPage = 64;         // tokens per page
-constexpr int kRows = 16;         // query-head rows per tile (G <= 16, zero-padded)
-constexpr int kConsumerWarps = 8; // two warpgroups
+constexpr int kPage = 64;          // tokens per page
+constexpr int kRows = 16;          // query-head rows per tile (G <= 16, zero-padded)
+constexpr int kConsumerWarps = 8;  // two warpgroups
 constexpr int kGroups = 2;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kChunkBytes = kPage * 64 * 2;  // one 64-column half of a page-head: 8 KiB
+constexpr int kChunkBytes = kPage * 64 * 2;  // one 64-column half of a bf16 page-head: 8 KiB
+constexpr int kMergeSlots = 2;               // 16 x D fp32 buffers for the cross-warp merge
 
-template <int D>
+enum KvFormat { kBF16 = 0, kNVFP4 = 1 };
+
+template <int D, int FMT>
 struct GqaCfg {
-  static constexpr int NCH = D / 64;                        // 64-column halves per row
-  static constexpr int STAGE_BYTES = 2 * NCH * kChunkBytes;  // K + V of one (page, kv head)
-  static constexpr int NSTAGE = (D == 128) ? 5 : 10;
+  static constexpr int NCH = D / 64;  // 64-column halves per bf16 row
+  // NVFP4 stage: K codes | K scales | V codes | V scales of one (page, kv head)
+  static constexpr int KC_BYTES = kPage * D / 2, KS_BYTES = kPage * D / 16;
+  static constexpr int OFF_KS = KC_BYTES, OFF_VC = KC_BYTES + KS_BYTES,
+                       OFF_VS = 2 * KC_BYTES + KS_BYTES;
+  static constexpr int STAGE_BYTES =
+      FMT == kBF16 ? 2 * NCH * kChunkBytes : 2 * (KC_BYTES + KS_BYTES);
+  static constexpr int NSTAGE = FMT == kNVFP4 ? 16 : (D == 128 ? 6 : 10);
   // floats per workspace segment record: O [16][D], then m, l, lb per row
   static constexpr int REC = kRows * (D + 3);
+  static_assert(NSTAGE % kGroups == 0, "a stage must belong to one consumer group");
+  static_assert(NSTAGE <= 16, "SmemTail holds 16 barrier pairs");
 };
 
 struct SmemTail {
   uint64_t full[16];
   uint64_t empty[16];
+  int stage_ok[16];  // written by the producer before it completes a stage: 1 = page loaded
   float mstat[kConsumerWarps][kRows];
   float lstat[kConsumerWarps][kRows];
   float lbstat[kConsumerWarps][kRows];
@@ -56,10 +83,10 @@ struct SmemTail {
   int abort_;
 };
 
-template <int D>
+template <int D, int FMT>
 __host__ __device__ constexpr size_t smem_bytes_for(int units) {
-  return 1024 /*alignment slack*/ + (size_t)GqaCfg<D>::NSTAGE * GqaCfg<D>::STAGE_BYTES +
-         4 * (size_t)kRows * D * sizeof(float) + sizeof(SmemTail) +
+  return 1024 /*alignment slack*/ + (size_t)GqaCfg<D, FMT>::NSTAGE * GqaCfg<D, FMT>::STAGE_BYTES +
+         (size_t)kMergeSlots * kRows * D * sizeof(float) + sizeof(SmemTail) +
          (size_t)(units + 1) * sizeof(int);
 }
 
@@ -71,18 +98,48 @@ __device__ __forceinline__ int cta_of(long long x, long long W, int G) {
   return (int)(((x + 1) * (long long)G - 1) / W);
 }
 
-// Warp-collective pipeline wait: lane 0 polls with a time limit, the result is broadcast.
+// Warp-collective pipeline wait: every lane observes the phase itself (so each lane's later shared
+// memory reads are ordered after the asynchronous writes the phase covers); false on timeout.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity);
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  const bool ok = mbar_wait(bar, parity);
+  return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
+// ---- NVFP4 helpers: hardware conversions of packed 4-/8-bit codes to f16x2 (low code -> low half)
+__device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t& h0, uint32_t& h1,
+                                                uint32_t& h2, uint32_t& h3) {
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "r"(w));
+}
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  return h;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float f16_lo_to_f32(uint32_t v) {
+  return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));
+}
+__device__ __forceinline__ float f16_hi_to_f32(uint32_t v) {
+  return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
+}
+
+template <int D, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
-    gqa_partial_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
-                            const __grid_constant__ CUtensorMap tmV, const GqaParams p) {
-  using Cfg = GqaCfg<D>;
+    gqa_partial_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const GqaParams p) {
+  using Cfg = GqaCfg<D, FMT>;
   constexpr int NCH = Cfg::NCH;
   constexpr int NSTAGE = Cfg::NSTAGE;
   constexpr int KSTEPS = D / 16;  // k-steps of the QK^T contraction
@@ -93,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* stages = smem;
   float* Obuf = reinterpret_cast<float*>(smem + (size_t)NSTAGE * Cfg::STAGE_BYTES);
-  SmemTail* tail = reinterpret_cast<SmemTail*>(Obuf + 4 * kRows * D);
+  SmemTail* tail = reinterpret_cast<SmemTail*>(Obuf + kMergeSlots * kRows * D);
   int* pre = reinterpret_cast<int*>(tail + 1);
 
   const int tid = threadIdx.x;
@@ -120,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < NSTAGE; ++i) {
       mbar_init(&tail->full[i], 1);
       mbar_init(&tail->empty[i], 4);
+      tail->stage_ok[i] = 0;
     }
     fence_mbar_init();
   }
@@ -170,56 +228,77 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ======================================= producer =============================================
   if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      int u = u_first;
-      long long i = 0;
-      int stage = 0;
-      uint32_t round = 0;
-      bool dead = false;
-      int s = 0, k = 0, b = 0;
-      const int32_t* ptab = nullptr;
-      int cur = -1;
-      for (long long g = g_begin; g < g_end; ++g, ++i) {
-        while (pre[u + 1] <= g) ++u;
-        if (u != cur) {
-          cur = u;
-          s = u % p.kvp;
-          const int bk = u / p.kvp;
-          k = bk % p.Hkv;
-          b = bk / p.Hkv;
-          ptab = p.page_table + ((size_t)s * p.B + b) * p.max_pages;
-        }
-        const int pg = (int)(g - pre[u]);
-        if (*(volatile int*)&tail->abort_) { dead = true; break; }
-        if (round > 0 && !mbar_wait(&tail->empty[stage], (round - 1) & 1)) {
-          raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
-          *(volatile int*)&tail->abort_ = 1;
-          dead = true;
-          break;
-        }
-        const int page = __ldg(ptab + pg);
-        if (page < 0 || page >= p.num_pages) {
-          raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
-          mbar_arrive(&tail->full[stage]);  // completes the phase with no data; consumers skip
-        } else {
-          uint8_t* st = stages + (size_t)stage * Cfg::STAGE_BYTES;
-          const int row = (page * p.Hkv + k) * kPage;
-          mbar_arrive_expect_tx(&tail->full[stage], Cfg::STAGE_BYTES);
+    if constexpr (FMT == kBF16) {
+      if (lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+      }
+    }
+    int u_cur = u_first;  // unit of the first page of the current batch (same in every lane)
+    int stage = 0;
+    uint32_t round = 0;
+    long long issued = 0;
+    bool dead = false;
+    for (long long gb = g_begin; gb < g_end && !dead; gb += 32) {
+      // each lane resolves page gb + lane: its unit, KV head and pool page id (one coalesced load)
+      const long long gl = gb + lane;
+      int my_page = -1, my_k = 0, uu = u_cur;
+      if (gl < g_end) {
+        while (pre[uu + 1] <= gl) ++uu;
+        const int s = uu % p.kvp, bk = uu / p.kvp, b = bk / p.Hkv;
+        my_k = bk % p.Hkv;
+        my_page = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + (int)(gl - pre[uu]));
+      }
+      const int nb = (int)min(32LL, g_end - gb);
+      u_cur = __shfl_sync(0xffffffffu, uu, nb - 1);
+      for (int j = 0; j < nb; ++j) {
+        const int page = __shfl_sync(0xffffffffu, my_page, j);
+        const int k = __shfl_sync(0xffffffffu, my_k, j);
+        if (lane == 0 && !dead) {
+          if (*(volatile int*)&tail->abort_) {
+            dead = true;
+          } else if (round > 0 && !mbar_wait(&tail->empty[stage], (round - 1) & 1)) {
+            raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
+            *(volatile int*)&tail->abort_ = 1;
+            dead = true;
+          } else {
+            uint8_t* st = stages + (size_t)stage * Cfg::STAGE_BYTES;
+            if (page < 0 || page >= p.num_pages) {
+              raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
+              tail->stage_ok[stage] = 0;
+              mbar_arrive(&tail->full[stage]);  // completes the phase with no data
+            } else {
+              tail->stage_ok[stage] = 1;
+              mbar_arrive_expect_tx(&tail->full[stage], Cfg::STAGE_BYTES);
+              if constexpr (FMT == kBF16) {
+                const int row = (page * p.Hkv + k) * kPage;
 #pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            tma_load_2d(st + c * kChunkBytes, &tmK, c * 64, row, &tail->full[stage]);
-            tma_load_2d(st + (NCH + c) * kChunkBytes, &tmV, c * 64, row, &tail->full[stage]);
+                for (int c = 0; c < NCH; ++c) {
+                  tma_load_2d(st + c * kChunkBytes, &tmK, c * 64, row, &tail->full[stage]);
+                  tma_load_2d(st + (NCH + c) * kChunkBytes, &tmV, c * 64, row,
+                              &tail->full[stage]);
+                }
+              } else {
+                const size_t ph = (size_t)page * p.Hkv + k;
+                bulk_load(st, p.k_codes + ph * Cfg::KC_BYTES, Cfg::KC_BYTES, &tail->full[stage]);
+                bulk_load(st + Cfg::OFF_KS, p.k_scale + ph * Cfg::KS_BYTES, Cfg::KS_BYTES,
+                          &tail->full[stage]);
+                bulk_load(st + Cfg::OFF_VC, p.v_codes + ph * Cfg::KC_BYTES, Cfg::KC_BYTES,
+                          &tail->full[stage]);
+                bulk_load(st + Cfg::OFF_VS, p.v_scale + ph * Cfg::KS_BYTES, Cfg::KS_BYTES,
+                          &tail->full[stage]);
+              }
+            }
+            ++issued;
+            if (++stage == NSTAGE) { stage = 0; ++round; }
           }
         }
-        if (++stage == NSTAGE) { stage = 0; ++round; }
+        dead = __shfl_sync(0xffffffffu, dead ? 1 : 0, 0) != 0;
       }
-      if (dead) {  // let every load already issued land before the CTA exits
-        const long long n_issued = i;
-        for (long long j = n_issued > NSTAGE ? n_issued - NSTAGE : 0; j < n_issued; ++j)
-          mbar_wait(&tail->full[j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
-      }
+    }
+    if (dead && lane == 0) {  // let every load already issued land before the CTA exits
+      for (long long j = issued > NSTAGE ? issued - NSTAGE : 0; j < issued; ++j)
+        mbar_wait(&tail->full[j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
     }
     return;
   }
@@ -234,9 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t qa[KSTEPS][4];
   float O[NT][4];
-  // m: running max (base-2 logits); l: sum of fp32 weights (for the LSE); lb: sum of the
-  // bf16-rounded weights the tensor cores multiply V by (normalises O, so O stays a convex
-  // combination of V rows to fp32 accuracy)
+  // m: running max (base-2 logits); l: sum of fp32 weights (for the LSE); lb: sum of the rounded
+  // weights the tensor cores multiply V by (normalises O, so O stays a convex combination of V rows)
   float m_run[2], l_run[2], lb_run[2];
   auto reset_state = [&]() {
 #pragma unroll
@@ -249,29 +327,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bk = u / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
     const __nv_bfloat16* qb = p.q + ((size_t)b * p.Hq + (size_t)k * p.G) * D;
     const bool v0 = g8 < p.G, v1 = g8 + 8 < p.G;
+    const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qb + (size_t)g8 * D);
+    const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qb + (size_t)(g8 + 8) * D);
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
-      const int c0 = 16 * kk + 2 * t4;
-      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qb + (size_t)g8 * D);
-      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qb + (size_t)(g8 + 8) * D);
-      qa[kk][0] = v0 ? __ldg(r0 + c0 / 2) : 0u;
-      qa[kk][1] = v1 ? __ldg(r1 + c0 / 2) : 0u;
-      qa[kk][2] = v0 ? __ldg(r0 + (c0 + 8) / 2) : 0u;
-      qa[kk][3] = v1 ? __ldg(r1 + (c0 + 8) / 2) : 0u;
+      if constexpr (FMT == kBF16) {
+        const int c0 = 16 * kk + 2 * t4;
+        qa[kk][0] = v0 ? __ldg(r0 + c0 / 2) : 0u;
+        qa[kk][1] = v1 ? __ldg(r1 + c0 / 2) : 0u;
+        qa[kk][2] = v0 ? __ldg(r0 + (c0 + 8) / 2) : 0u;
+        qa[kk][3] = v1 ? __ldg(r1 + (c0 + 8) / 2) : 0u;
+      } else {
+        // permuted k: logical columns (2t, 2t+1 | 2t+8, 2t+9) of k-step kk are head-dim elements
+        // 32t + 4kk + (0, 1 | 2, 3); q is rounded to f16 (exact for |q| >= 2^-14)
+        const int c0 = 32 * t4 + 4 * kk;
+        auto cvt = [](uint32_t bf2) {  // bf16x2 -> f16x2
+          return pack_f16x2(bf16_lo_to_f32(bf2), bf16_hi_to_f32(bf2));
+        };
+        qa[kk][0] = v0 ? cvt(__ldg(r0 + c0 / 2)) : 0u;
+        qa[kk][1] = v1 ? cvt(__ldg(r1 + c0 / 2)) : 0u;
+        qa[kk][2] = v0 ? cvt(__ldg(r0 + c0 / 2 + 1)) : 0u;
+        qa[kk][3] = v1 ? cvt(__ldg(r1 + c0 / 2 + 1)) : 0u;
+      }
     }
   };
 
   reset_state();
   int u = u_first;
   int s_u = 0, b_u = 0, k_u = 0, len_u = 0;
-  const int32_t* ptab = nullptr;
   auto enter_unit = [&](int uu) {
     s_u = uu % p.kvp;
     const int bk = uu / p.kvp;
     k_u = bk % p.Hkv;
     b_u = bk / p.Hkv;
     len_u = p.shard_lens[s_u * p.B + b_u];
-    ptab = p.page_table + ((size_t)s_u * p.B + b_u) * p.max_pages;
     load_q(uu);
   };
   enter_unit(u);
@@ -296,28 +385,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         dead = true;
       }
       if (!dead) {
-        const int page = __ldg(ptab + pg);
         const int nvalid = min(kPage, len_u - pg * kPage);
         uint8_t* st = stages + (size_t)stage * Cfg::STAGE_BYTES;
-        const bool page_ok = page >= 0 && page < p.num_pages;
-        if (page_ok && tok0 < nvalid) {
-          const uint32_t kbase = smem_u32(st);
-          const uint32_t vbase = kbase + NCH * kChunkBytes;
-          // zero the V rows past the end of the history in this warp's slice (0 * garbage = NaN)
-          if (tok0 + 16 > nvalid) {
-            for (int e = lane; e < 16 * NCH * 8; e += 32) {
-              const int row = tok0 + e / (NCH * 8);
-              const int rem = e % (NCH * 8);
-              if (row >= nvalid)
-                *reinterpret_cast<uint4*>(st + (NCH + rem / 8) * kChunkBytes + row * 128 +
-                                          (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-          }
-          // S = q K^T over this warp's 16 tokens: two n-tiles of 8 tokens
+        if (tail->stage_ok[stage] && tok0 < nvalid) {
           float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-          {
+          if constexpr (FMT == kBF16) {
+            const uint32_t kbase = smem_u32(st);
+            // zero the V rows past the end of the history in this warp's slice (0 * garbage = NaN)
+            if (tok0 + 16 > nvalid) {
+              for (int e = lane; e < 16 * NCH * 8; e += 32) {
+                const int row = tok0 + e / (NCH * 8);
+                const int rem = e % (NCH * 8);
+                if (row >= nvalid)
+                  *reinterpret_cast<uint4*>(st + (NCH + rem / 8) * kChunkBytes + row * 128 +
+                                            (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+            }
+            // S = q K^T over this warp's 16 tokens: two n-tiles of 8 tokens
             const int token = tok0 + (mi >> 1) * 8 + r8;
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -329,6 +415,26 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_bf16_16816(s0, qa[kk], b0, b1);
               mma_bf16_16816(s1, qa[kk], b2, b3);
             }
+          } else {
+            // S = q K^T from NVFP4: token g8 of each n-tile, head-dim elements [32 t4, 32 t4 + 32)
+            auto ntile = [&](float(&acc)[4], int token) {
+              const uint4 kc = *reinterpret_cast<const uint4*>(st + token * (D / 2) + t4 * 16);
+              const uint32_t sc2 = e4m3x2_to_f16x2(
+                  *reinterpret_cast<const uint16_t*>(st + Cfg::OFF_KS + token * (D / 16) + 2 * t4));
+              const uint32_t sc_lo = __byte_perm(sc2, 0, 0x1010);  // (s_2t, s_2t)
+              const uint32_t sc_hi = __byte_perm(sc2, 0, 0x3232);  // (s_2t+1, s_2t+1)
+              const uint32_t words[4] = {kc.x, kc.y, kc.z, kc.w};
+#pragma unroll
+              for (int wq = 0; wq < 4; ++wq) {  // word wq holds k-steps 2wq and 2wq+1
+                uint32_t h0, h1, h2, h3;
+                e2m1x4_to_f16x2(words[wq], h0, h1, h2, h3);
+                const uint32_t sc = wq < 2 ? sc_lo : sc_hi;
+                mma_f16_16816(acc, qa[2 * wq], hmul2(h0, sc), hmul2(h1, sc));
+                mma_f16_16816(acc, qa[2 * wq + 1], hmul2(h2, sc), hmul2(h3, sc));
+              }
+            };
+            ntile(s0, tok0 + g8);
+            ntile(s1, tok0 + 8 + g8);
           }
           // online softmax (base 2)
           const int ta = tok0 + 2 * t4, tb = tok0 + 8 + 2 * t4;
@@ -358,17 +464,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) pw[e] = fast_exp2(x[e] - mu0);
 #pragma unroll
           for (int e = 4; e < 8; ++e) pw[e] = fast_exp2(x[e] - mu1);
-          uint32_t pa[4];
-          pa[0] = pack_bf16x2(pw[0], pw[1]);  // row g,   k 2t..
-          pa[1] = pack_bf16x2(pw[4], pw[5]);  // row g+8, k 2t..
-          pa[2] = pack_bf16x2(pw[2], pw[3]);  // row g,   k 8+2t..
-          pa[3] = pack_bf16x2(pw[6], pw[7]);  // row g+8, k 8+2t..
           l_run[0] = l_run[0] * al0 + ((pw[0] + pw[1]) + (pw[2] + pw[3]));
           l_run[1] = l_run[1] * al1 + ((pw[4] + pw[5]) + (pw[6] + pw[7]));
-          lb_run[0] = lb_run[0] * al0 + (bf16_lo_to_f32(pa[0]) + bf16_hi_to_f32(pa[0])) +
-                      (bf16_lo_to_f32(pa[2]) + bf16_hi_to_f32(pa[2]));
-          lb_run[1] = lb_run[1] * al1 + (bf16_lo_to_f32(pa[1]) + bf16_hi_to_f32(pa[1])) +
-                      (bf16_lo_to_f32(pa[3]) + bf16_hi_to_f32(pa[3]));
+          uint32_t pa[4];
+          if constexpr (FMT == kBF16) {
+            pa[0] = pack_bf16x2(pw[0], pw[1]);  // row g,   k 2t..
+            pa[1] = pack_bf16x2(pw[4], pw[5]);  // row g+8, k 2t..
+            pa[2] = pack_bf16x2(pw[2], pw[3]);  // row g,   k 8+2t..
+            pa[3] = pack_bf16x2(pw[6], pw[7]);  // row g+8, k 8+2t..
+            lb_run[0] = lb_run[0] * al0 + (bf16_lo_to_f32(pa[0]) + bf16_hi_to_f32(pa[0])) +
+                        (bf16_lo_to_f32(pa[2]) + bf16_hi_to_f32(pa[2]));
+            lb_run[1] = lb_run[1] * al1 + (bf16_lo_to_f32(pa[1]) + bf16_hi_to_f32(pa[1])) +
+                        (bf16_lo_to_f32(pa[3]) + bf16_hi_to_f32(pa[3]));
+          } else {
+            pa[0] = pack_f16x2(pw[0], pw[1]);
+            pa[1] = pack_f16x2(pw[4], pw[5]);
+            pa[2] = pack_f16x2(pw[2], pw[3]);
+            pa[3] = pack_f16x2(pw[6], pw[7]);
+            lb_run[0] = lb_run[0] * al0 + (f16_lo_to_f32(pa[0]) + f16_hi_to_f32(pa[0])) +
+                        (f16_lo_to_f32(pa[2]) + f16_hi_to_f32(pa[2]));
+            lb_run[1] = lb_run[1] * al1 + (f16_lo_to_f32(pa[1]) + f16_hi_to_f32(pa[1])) +
+                        (f16_lo_to_f32(pa[3]) + f16_hi_to_f32(pa[3]));
+          }
           if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
@@ -378,8 +495,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               O[j][3] *= al1;
             }
           }
-          // O += P V over the 16 tokens: V^T fragments via transposing ldmatrix
-          {
+          if constexpr (FMT == kBF16) {
+            // O += P V over the 16 tokens: V^T fragments via transposing ldmatrix
+            const uint32_t vbase = smem_u32(st) + NCH * kChunkBytes;
             const int token = tok0 + (mi & 1) * 8 + r8;
 #pragma unroll
             for (int n2 = 0; n2 < NT / 2; ++n2) {
@@ -390,6 +508,36 @@ __global__ void __launch_bounds__(kThreads, 1)
               ldsm_x4_trans(addr, v0, v1, v2, v3);
               mma_bf16_16816(O[2 * n2], pa, v0, v1);
               mma_bf16_16816(O[2 * n2 + 1], pa, v2, v3);
+            }
+          } else {
+            // O += P V from NVFP4: token pairs (2t, 2t+1) and (2t+8, 2t+9) of the slice, output
+            // columns 16 g8 + j (n-tile j). A pair row's 16-byte chunks are stored XOR-swizzled by
+            // 2 (pair mod 4), which spreads the eight lanes of a quarter-warp over all banks. The
+            // scales of tokens past the history are zeroed so their codes contribute nothing.
+            const uint8_t* vc = st + Cfg::OFF_VC;
+            const uint8_t* vsc = st + Cfg::OFF_VS + g8 * kPage;
+            const int pa_ = tok0 / 2 + t4, pb_ = tok0 / 2 + t4 + 4;
+            const uint4 va = *reinterpret_cast<const uint4*>(vc + pa_ * D +
+                                                             ((g8 ^ ((pa_ & 3) << 1)) << 4));
+            const uint4 vb = *reinterpret_cast<const uint4*>(vc + pb_ * D +
+                                                             ((g8 ^ ((pb_ & 3) << 1)) << 4));
+            uint32_t sa = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc + ta));
+            uint32_t sb = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc + tb));
+            const uint32_t ma = (ta < nvalid ? 0x0000ffffu : 0u) | (ta + 1 < nvalid ? 0xffff0000u : 0u);
+            const uint32_t mb = (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
+            sa &= ma;
+            sb &= mb;
+            const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+            const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+            for (int wq = 0; wq < 4; ++wq) {
+              uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+              e2m1x4_to_f16x2(wa[wq], a0, a1, a2, a3);
+              e2m1x4_to_f16x2(wb[wq], c0, c1, c2, c3);
+              mma_f16_16816(O[4 * wq + 0], pa, hmul2(a0, sa), hmul2(c0, sb));
+              mma_f16_16816(O[4 * wq + 1], pa, hmul2(a1, sa), hmul2(c1, sb));
+              mma_f16_16816(O[4 * wq + 2], pa, hmul2(a2, sa), hmul2(c2, sb));
+              mma_f16_16816(O[4 * wq + 3], pa, hmul2(a3, sa), hmul2(c3, sb));
             }
           }
         }
@@ -439,8 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           O[j][3] *= a1;
         }
       }
-      // Sum the 8 warps' O in a fixed order (4+4, 2+2, 1+1) so results are bit-reproducible.
-      // Four 16 x D buffers; every warp only overwrites a buffer it has finished reading itself.
+      // Sum the 8 warps' O in a fixed order so results are bit-reproducible: warps 4..7 into
+      // 0..3 (two at a time through the two merge slots), then 2,3 into 0,1, then 1 into 0.
       {
         auto put = [&](int slot) {
           float* dst = Obuf + slot * kRows * D;
@@ -456,26 +604,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) O[j][e] += src[(j * 4 + e) * 32 + lane];
         };
-        if (cw >= 4) put(cw - 4);
+        // (writer warps, reader warps): (4,5 -> 0,1), (6,7 -> 2,3), (2,3 -> 0,1), (1 -> 0)
+        if (cw == 4 || cw == 5) put(cw - 4);
         named_barrier_sync(1, kConsumerWarps * 32);
-        if (cw < 4) add(cw);
-        __syncwarp();
-        if (cw == 2 || cw == 3) put(cw);
+        if (cw == 0 || cw == 1) add(cw);
         named_barrier_sync(1, kConsumerWarps * 32);
-        if (cw < 2) add(cw + 2);
-        __syncwarp();
+        if (cw == 6 || cw == 7) put(cw - 6);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (cw == 2 || cw == 3) add(cw - 2);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (cw == 2 || cw == 3) put(cw - 2);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (cw == 0 || cw == 1) add(cw);
+        named_barrier_sync(1, kConsumerWarps * 32);
         if (cw == 1) put(1);
         named_barrier_sync(1, kConsumerWarps * 32);
         if (cw == 0) {
           add(1);
-          __syncwarp();
 #pragma unroll
-          for (int j = 0; j < NT; ++j) {  // natural [row][column] layout for the output phase
-            float* r0 = Obuf + g8 * D + 8 * j + 2 * t4;
-            r0[0] = O[j][0];
-            r0[1] = O[j][1];
-            r0[8 * D] = O[j][2];
-            r0[8 * D + 1] = O[j][3];
+          for (int j = 0; j < NT; ++j) {  // natural [row][column] layout into slot 0
+            // n-tile j, fragment columns 2t, 2t+1 are head-dim columns 8j + 2t (+1) for bf16 and
+            // 16 (2t) + j, 16 (2t + 1) + j for NVFP4 (its permuted n index)
+            const int ca = FMT == kBF16 ? 8 * j + 2 * t4 : 32 * t4 + j;
+            const int cb = FMT == kBF16 ? ca + 1 : 32 * t4 + 16 + j;
+            float* r0 = Obuf + g8 * D;
+            r0[ca] = O[j][0];
+            r0[cb] = O[j][1];
+            r0[8 * D + ca] = O[j][2];
+            r0[8 * D + cb] = O[j][3];
           }
         }
       }
@@ -511,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const int slot = (g_begin >= pre[u]) ? 0 : 1;
-        float* rec = p.seg + ((size_t)blockIdx.x * 2 + slot) * GqaCfg<D>::REC;
+        float* rec = p.seg + ((size_t)blockIdx.x * 2 + slot) * Cfg::REC;
 #pragma unroll
         for (int c = 0; c < D / 16; c += 4) {
           *reinterpret_cast<float4*>(rec + r * D + c0 + c) =
@@ -537,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float Mm = -INFINITY;
           for (int c = c_lo; c <= c_hi; ++c) {
             const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
-            const float* rc = p.seg + ((size_t)c * 2 + sl) * GqaCfg<D>::REC;
+            const float* rc = p.seg + ((size_t)c * 2 + sl) * Cfg::REC;
             Mm = fmaxf(Mm, __ldcg(rc + kRows * D + r));
           }
           const float Mmu = Mm == -INFINITY ? 0.f : Mm;
@@ -547,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float Lm = 0.f, LBm = 0.f;
           for (int c = c_lo; c <= c_hi; ++c) {
             const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
-            const float* rc = p.seg + ((size_t)c * 2 + sl) * GqaCfg<D>::REC;
+            const float* rc = p.seg + ((size_t)c * 2 + sl) * Cfg::REC;
             const float wgt = fast_exp2(__ldcg(rc + kRows * D + r) - Mmu);
             Lm += __ldcg(rc + kRows * D + kRows + r) * wgt;
             LBm += __ldcg(rc + kRows * D + 2 * kRows + r) * wgt;
@@ -581,11 +737,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D>
-static helix_status launch_bf16(const CUtensorMap& tmK, const CUtensorMap& tmV,
-                                const GqaParams& p, int grid, cudaStream_t stream) {
-  const size_t smem = smem_bytes_for<D>(p.units);
-  auto kern = gqa_partial_bf16_kernel<D>;
+template <int D, int FMT>
+static helix_status launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const GqaParams& p,
+                           int grid, cudaStream_t stream) {
+  const size_t smem = smem_bytes_for<D, FMT>(p.units);
+  auto kern = gqa_partial_kernel<D, FMT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return HELIX_ERR_CUDA;
@@ -593,19 +749,26 @@ static helix_status launch_bf16(const CUtensorMap& tmK, const CUtensorMap& tmV,
   return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
 }
 
-size_t gqa_partial_smem_bytes(int head_dim, int units) {
-  return head_dim == 64 ? smem_bytes_for<64>(units) : smem_bytes_for<128>(units);
+size_t gqa_partial_smem_bytes(int head_dim, int nvfp4, int units) {
+  if (nvfp4) return smem_bytes_for<128, kNVFP4>(units);
+  return head_dim == 64 ? smem_bytes_for<64, kBF16>(units) : smem_bytes_for<128, kBF16>(units);
 }
 
 size_t gqa_segment_record_floats(int head_dim) {
-  return head_dim == 64 ? GqaCfg<64>::REC : GqaCfg<128>::REC;
+  return head_dim == 64 ? GqaCfg<64, kBF16>::REC : GqaCfg<128, kBF16>::REC;
 }
 
 helix_status gqa_partial_bf16_launch(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                      const GqaParams& p, int grid, cudaStream_t stream) {
-  if (p.D == 128) return launch_bf16<128>(tmK, tmV, p, grid, stream);
-  if (p.D == 64) return launch_bf16<64>(tmK, tmV, p, grid, stream);
+  if (p.D == 128) return launch<128, kBF16>(tmK, tmV, p, grid, stream);
+  if (p.D == 64) return launch<64, kBF16>(tmK, tmV, p, grid, stream);
   return HELIX_ERR_UNSUPPORTED;
+}
+
+helix_status gqa_partial_nvfp4_launch(const GqaParams& p, int grid, cudaStream_t stream) {
+  if (p.D != 128) return HELIX_ERR_UNSUPPORTED;
+  CUtensorMap unused{};
+  return launch<128, kNVFP4>(unused, unused, p, grid, stream);
 }
 
 }  // namespace helix

@@ -29,10 +29,11 @@ struct GqaParams {
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-size_t gqa_partial_smem_bytes(int head_dim, int units);
+size_t gqa_partial_smem_bytes(int head_dim, int nvfp4, int units);
 size_t gqa_segment_record_floats(int head_dim);
 helix_status gqa_partial_bf16_launch(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                      const GqaParams& p, int grid, cudaStream_t stream);
+helix_status gqa_partial_nvfp4_launch(const GqaParams& p, int grid, cudaStream_t stream);
 
 // Append: copies the new tokens' rows (and scales) into their pages.
 struct AppendParams {
@@ -44,6 +45,7 @@ struct AppendParams {
   int32_t* seq_lens;
   uint32_t* err;
   const int32_t* n_valid;  // optional [B]
+  int v_nvfp4;             // 1: streams 1 and 3 (V codes, V scales) use the token-pair layout
   int B, Hkv, kvp, layout, rr_block, contig_chunk, page_tokens, max_pages, num_pages, n_new;
 };
 helix_status append_launch(const AppendParams& p, cudaStream_t stream);

@@ -55,19 +55,29 @@ def test_append_bit_exact(cfg):
     assert cache["shard_lens"].t().tolist() == want_shards
     if w.kind == "mla":
         _expected_pool(w, cache, [allrows["k_new"][b].cpu() for b in range(w.B)], lens, "k")
-    else:
+    elif w.kv_dtype == "bf16":
         for st, key in (("k", "k_new"), ("v", "v_new")):
             _expected_pool(w, cache, [allrows[key][b].cpu() for b in range(w.B)], lens, st)
-        if w.kv_dtype == "nvfp4":
-            for st, key in (("k_scale", "k_scale"), ("v_scale", "v_scale")):
-                pool = cache[st].cpu()
-                pt = cache.page_table.cpu()
-                for b in range(w.B):
-                    for t in range(lens[b]):
-                        s, l_ = oracle.rr_place(t, w.kvp, w.rr_block)
-                        pi, slot = oracle.page_slot(l_)
-                        assert torch.equal(pool[int(pt[s, b, pi]), :, slot],
-                                           allrows[key][b, t].cpu())
+    else:
+        # K codes and K scales: natural rows. V codes: byte [slot // 2][c] holds element c of the
+        # token in nibble slot % 2. V scales: [block][slot].
+        _expected_pool(w, cache, [allrows["k_new"][b].cpu() for b in range(w.B)], lens, "k")
+        ks, vp, vs = cache["k_scale"].cpu(), cache["v_pool"].cpu(), cache["v_scale"].cpu()
+        pt = cache.page_table.cpu()
+        for b in range(w.B):
+            for t in range(lens[b]):
+                s, l_ = oracle.rr_place(t, w.kvp, w.rr_block)
+                pi, slot = oracle.page_slot(l_)
+                page = int(pt[s, b, pi])
+                assert torch.equal(ks[page, :, slot], allrows["k_scale"][b, t].cpu())
+                assert torch.equal(vs[page, :, :, slot], allrows["v_scale"][b, t].cpu())
+                src = allrows["v_new"][b, t].cpu().to(torch.int32)  # [H, d/2] natural packing
+                codes = torch.stack([src & 0xF, src >> 4], -1).reshape(w.Hkv, w.d)
+                pair = slot // 2
+                col = torch.arange(w.d)
+                pos = 16 * ((col // 16) ^ (2 * (pair % 4))) + col % 16  # documented swizzle
+                got = (vp[page, :, pair, :][:, pos].to(torch.int32) >> (4 * (slot % 2))) & 0xF
+                assert torch.equal(got, codes), (b, t)
 
 
 def test_append_capacity_and_bad_page_errors():

@@ -50,6 +50,16 @@ SMALL = {
 }
 
 
+NVFP4 = wl.WORKLOADS["gqa_nvfp4_s1m"]
+SMALL.update({
+    # NVFP4 KV: ragged lengths with G=16, empty shards, and units split across CTAs
+    "nvfp4_rr_ragged": (NVFP4.with_(B=3, Hq=48, Hkv=3, S=3000), [3000, 1, 77]),
+    "nvfp4_empty_shards": (NVFP4.with_(B=2, Hq=16, Hkv=2, S=40), [40, 17]),
+    "nvfp4_split_units": (NVFP4.with_(B=1, Hq=8, Hkv=2, S=70000, kvp=2), [70000]),
+    "nvfp4_g4": (NVFP4.with_(B=2, Hq=16, Hkv=4, S=2500, kvp=3), [2500, 1300]),
+})
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_gqa_small(name):
     w, lens = SMALL[name]
@@ -58,6 +68,18 @@ def test_gqa_small(name):
     assert cache.err_bits() == 0
     q = wl.query(w, "cuda")
     _check_all_heads(w, q, lens, _run(cache, w, q), name)
+
+
+def test_gqa_nvfp4_sharp():
+    """NVFP4 KV with a sharp query (q x 8): near one-hot softmax, |O| of order |V|."""
+    w = NVFP4.with_(B=2, Hq=32, Hkv=2, S=5000)
+    lens = [5000, 4321]
+    cache = _gpu.make_cache(w)
+    _gpu.fill(cache, w, lens, chunk=2048)
+    q = wl.query(w, "cuda", scale_by=8.0)
+    res = _run(cache, w, q)
+    _check_all_heads(w, q, lens, res, "nvfp4 sharp")
+    assert np.abs(res[2]).max() > 0.3
 
 
 @pytest.mark.parametrize("kind", ["sharp", "needle", "shift"])
@@ -129,6 +151,29 @@ def test_gqa_repeat_is_deterministic_and_tickets_reset():
     assert int(ws[: 4 * w.B * w.Hkv * w.kvp].view(torch.int32).abs().sum()) == 0
 
 
+@pytest.mark.parametrize("kv_dtype", ["bf16", "nvfp4"])
+def test_gqa_repeat_variable_lengths_bit_identical(kv_dtype):
+    """Ragged lengths (a partial last page in every unit), many split units, several calls: the
+    results must not depend on the order in which pages land or warps finish."""
+    base = wl.WORKLOADS["gqa_s1m_var" if kv_dtype == "bf16" else "gqa_nvfp4_s1m"]
+    w = base.with_(B=8, Hq=32, Hkv=2, S=150000, S_min=None)
+    g = torch.Generator().manual_seed(11)
+    lens = [int(x) for x in torch.randint(40000, 150001, (w.B,), generator=g)]
+    cache = _gpu.make_cache(w)
+    _gpu.fill(cache, w, lens, chunk=16384)
+    q = wl.query(w, "cuda")
+    first = _run(cache, w, q)
+    for _ in range(3):
+        again = _run(cache, w, q)
+        for x, y in zip(first, again):
+            assert np.array_equal(x, y)
+    for b, h in ((int(np.argmin(lens)), 0), (int(np.argmax(lens)), 1)):
+        O, L, Os, Ls = _gpu.oracle_head_group(w, q, b, h, lens[b])
+        hs = slice(h * w.G, (h + 1) * w.G)
+        _gpu.assert_close_O(first[2][b, hs], O, f"O b={b}")
+        _gpu.assert_close_lse(first[3][b, hs], L, f"LSE b={b}")
+
+
 def test_gqa_bad_page_id_sets_error_and_skips():
     w = wl.WORKLOADS["gqa_s128k"].with_(B=1, Hq=16, Hkv=1, S=640, kvp=2)
     cache = _gpu.make_cache(w)
@@ -176,6 +221,11 @@ def test_gqa_full_128k_sampled():
 def test_gqa_full_1m_sampled():
     w = wl.WORKLOADS["gqa_s1m"]
     _sampled(w, wl.seq_lens(w), [(0, 0), (6, 3)])
+
+
+def test_gqa_nvfp4_full_1m_sampled():
+    w = wl.WORKLOADS["gqa_nvfp4_s1m"]
+    _sampled(w, wl.seq_lens(w), [(0, 0), (5, 6)])
 
 
 def test_gqa_full_1m_variable_sampled():
