@@ -119,8 +119,21 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
   helix_status st = check_cache(c);
   if (st != HELIX_OK) return st;
   if (num_q_heads < 1 || num_q_heads % c->num_kv_heads != 0) return HELIX_ERR_INVALID_ARG;
-  if (c->kind != HELIX_ATTN_GQA) return HELIX_ERR_UNSUPPORTED;
   if (c->page_tokens != 64) return HELIX_ERR_UNSUPPORTED;
+  if (c->kind == HELIX_ATTN_MLA) {
+    // one kernel shape: 128 heads against a 576-wide latent whose first 512 columns are V
+    if (num_q_heads != 128 || c->head_dim != 576 || c->v_dim != 512) return HELIX_ERR_UNSUPPORTED;
+    int sms = 0, max_smem = 0;
+    if (device_sm_count(&sms) != 0 || device_max_smem(&max_smem) != 0) return HELIX_ERR_CUDA;
+    plan->units = c->batch * c->kvp;
+    if (mla_partial_smem_bytes(plan->units) > (size_t)max_smem) return HELIX_ERR_CAPACITY;
+    plan->grid = (sms / 2) * 2;  // clusters of two CTAs
+    if (plan->grid < 2) return HELIX_ERR_UNSUPPORTED;
+    plan->ticket_bytes = (((size_t)plan->units * 2 * sizeof(int32_t)) + 255) & ~size_t(255);
+    plan->seg_bytes = (size_t)(plan->grid / 2) * 2 * 2 * mla_segment_record_floats() * sizeof(float);
+    return HELIX_OK;
+  }
+  if (c->kind != HELIX_ATTN_GQA) return HELIX_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return HELIX_ERR_UNSUPPORTED;
   if (num_q_heads / c->num_kv_heads > 16) return HELIX_ERR_UNSUPPORTED;
   const int nvfp4 = c->kv_dtype == HELIX_KV_NVFP4;
@@ -226,6 +239,32 @@ helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t 
     return HELIX_ERR_INVALID_ARG;
   if (workspace_bytes < plan.ticket_bytes + plan.seg_bytes) return HELIX_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return HELIX_ERR_INVALID_ARG;
+
+  if (c->kind == HELIX_ATTN_MLA) {
+    MlaParams m{};
+    m.page_table = c->page_table;
+    m.shard_lens = c->shard_lens;
+    m.o_part = o_partial;
+    m.lse = lse;
+    m.tickets = reinterpret_cast<int32_t*>(workspace);
+    m.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes);
+    m.err = c->err_word;
+    m.B = c->batch;
+    m.kvp = c->kvp;
+    m.max_pages = c->max_pages_per_shard;
+    m.num_pages = c->num_pages;
+    m.units = plan.units;
+    m.scale_log2 = softmax_scale * 1.4426950408889634f;
+    // latent pool as [pages * 64 rows][576], boxes of 64 columns x 32 rows; q as [B * 128][576],
+    // boxes of 64 columns x 128 rows; 128-byte swizzle for the tensor-core operand layout
+    CUtensorMap tmC, tmQ;
+    if (!encode_rows_map(&tmC, c->k_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
+                         (uint64_t)c->num_pages * 64, 64, 32) ||
+        !encode_rows_map(&tmQ, const_cast<void*>(q), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
+                         (uint64_t)c->batch * 128, 64, 128))
+      return HELIX_ERR_CUDA;
+    return mla_partial_launch(tmC, tmQ, m, plan.grid, reinterpret_cast<cudaStream_t>(stream));
+  }
 
   GqaParams p{};
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);

@@ -35,6 +35,23 @@ helix_status gqa_partial_bf16_launch(const CUtensorMap& tmK, const CUtensorMap& 
                                      const GqaParams& p, int grid, cudaStream_t stream);
 helix_status gqa_partial_nvfp4_launch(const GqaParams& p, int grid, cudaStream_t stream);
 
+// Parameters of the MLA partial kernel (128 heads, one 576-wide latent head, values = first 512).
+struct MlaParams {
+  const int32_t* page_table;  // [kvp][B][max_pages]
+  const int32_t* shard_lens;  // [kvp][B]
+  float* o_part;              // [kvp][B][128][512]
+  float* lse;                 // [kvp][B][128]
+  int32_t* tickets;           // [units][2], zero between launches
+  float* seg;                 // [clusters][2 slots][2 halves][record]
+  uint32_t* err;              // may be null
+  int B, kvp, max_pages, num_pages, units;
+  float scale_log2;
+};
+size_t mla_partial_smem_bytes(int units);
+size_t mla_segment_record_floats();
+helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmQ,
+                                const MlaParams& p, int grid, cudaStream_t stream);
+
 // Append: copies the new tokens' rows (and scales) into their pages.
 struct AppendParams {
   const uint8_t* src[4];   // k rows, v rows, k scales, v scales (null when unused)

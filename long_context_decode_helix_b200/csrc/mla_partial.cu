@@ -1,0 +1,673 @@
+// mla_partial.cu -- per-shard partial decode attention for absorbed multi-head latent attention
+// (MLA) on the 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
+//
+// What it computes: 128 query heads attend to ONE shared latent KV head (the paper summary's
+// tensor-parallelism paragraph notes that MLA "effectively" has one KV head, which is why its KV
+// cannot be split by heads and KV parallelism is needed). With the absorbed formulation the latent
+// row c_t (576 wide) is the key and its first 512 columns are the value:
+//     z_{h,t} = scale * <q_h, c_t>,  O_s[h] = sum_t e^{z - m} c_t[0:512] / sum_t e^{z - m},
+//     lse_s[h] = m + ln sum_t e^{z - m}
+// over the tokens T_s of KVP shard s (paper summary, paragraph on KV parallelism).
+//
+// Sizes force a two-CTA design. O for 128 heads x 512 columns in fp32 fills all 512 TMEM columns
+// and q (128 x 576 bf16) alone is 144 KiB, so one CTA cannot hold q, a score tile and O. A cluster
+// of two CTAs works on the same 32-token tiles:
+//   * CTA r keeps half of q's contraction (head-dim elements [288 r, 288 r + 288)) in shared memory
+//     and computes a partial score tile S_r = q[:, half] C[:, half]^T (M = 128 heads, N = 32 tokens,
+//     K = 288) into TMEM;
+//   * the two CTAs swap their partials through distributed shared memory (plain remote stores and
+//     remote mbarrier arrivals -- no multicast loads), so both hold the same full S;
+//   * each CTA runs the same online softmax and accumulates O for its half of the value columns
+//     (M = 128, N = 256, K = 32 tokens) in 256 TMEM columns, reading V straight from the latent tile
+//     it already holds (MN-major operand).
+// Each CTA loads five 64-column chunks of every latent row (chunks 0-4 or 4-8), so together the pair
+// reads the 576-wide row once plus one 64-column chunk.
+//
+// Warps: 0-3 softmax / epilogue (thread i owns head i = TMEM lane i), 4 TMA producer, 5 MMA issuer
+// (one elected thread) and TMEM allocator. O is rescaled lazily: the exponent base only moves when
+// a row maximum grows by more than 8 (in base-2 units), so weights stay below 2^8 and the 256-column
+// TMEM rescale is rare. Work is split over the (request, shard) units exactly as in the GQA kernel:
+// each cluster takes an equal contiguous range of 32-token tiles; split units are merged by the last
+// arriving cluster, per value half.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "device_common.cuh"
+#include "internal.h"
+
+namespace helix {
+namespace {
+
+constexpr int kHeads = 128;
+constexpr int kDK = 576, kDV = 512, kHalfDV = 256;
+constexpr int kTok = 32;                   // tokens per tile
+constexpr int kPageTok = 64;               // tokens per page
+constexpr int kChunks = 5;                 // 64-column chunks of a latent row per CTA
+constexpr int kKSteps = 18;                // 288 / 16
+constexpr int kNS = 4;                     // tile stages
+constexpr int kStageBytes = kTok * kChunks * 128;     // 20 KiB
+constexpr int kQBytes = kHeads * kChunks * 128;        // 80 KiB
+constexpr int kPBytes = kHeads * kTok * 2;             // 8 KiB (bf16 P tile, 64-byte rows)
+constexpr int kXStride = kTok + 4;                     // padded fp32 row of the exchange buffer
+constexpr int kXBytes = kHeads * kXStride * 4;         // 18 KiB
+constexpr int kThreads = 6 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kRec = kHeads * (kHalfDV + 3);           // floats per segment record (one half)
+
+struct MlaTail {
+  uint64_t stage_full[kNS], stage_empty[kNS];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t x_full[2], x_free[2];
+  uint64_t q_full, q_empty;
+  int stage_ok[kNS];
+  uint32_t tmem_base;
+  int flag;
+  int abort_;
+};
+
+constexpr size_t kSmemFixed = 1024 + kQBytes + kNS * kStageBytes + 2 * kPBytes + 2 * kXBytes +
+                              sizeof(MlaTail);
+
+// ------------------------------------------------------------------------------------------------
+// tcgen05 / cluster helpers
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// shared::cluster address of the same variable in CTA `rank`
+__device__ __forceinline__ uint32_t map_peer(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_bar_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   cluster_bar_addr)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+// wait with cluster-scope acquire (data written by the peer CTA)
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (sm_100 format): start, leading and stride byte offsets in
+// 16-byte units, descriptor version 1, swizzle mode in the top three bits.
+constexpr uint64_t kSwizzle128 = 2, kSwizzle64 = 4;
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint64_t swizzle) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (swizzle << 61);
+}
+// Instruction descriptor for kind::f16: fp32 accumulate, bf16 A and B, A K-major, B K-major or
+// MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ long long range_begin(int c, long long W, int G) {
+  return (long long)c * W / G;
+}
+__device__ __forceinline__ int cta_of(long long x, long long W, int G) {
+  return (int)(((x + 1) * (long long)G - 1) / W);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    mla_partial_kernel(const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ CUtensorMap tmQ, const MlaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* q_s = smem;                                   // [5 chunks][128 rows][128 B]
+  uint8_t* stage_s = q_s + kQBytes;                      // [kNS][5 chunks][32 rows][128 B]
+  uint8_t* p_s = stage_s + kNS * kStageBytes;            // [2][128 rows][64 B]
+  float* x_s = reinterpret_cast<float*>(p_s + 2 * kPBytes);  // [2][128][kXStride]
+  MlaTail* tail = reinterpret_cast<MlaTail*>(x_s + 2 * kHeads * kXStride);
+  int* pre = reinterpret_cast<int*>(tail + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer = rank ^ 1u;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int U = p.units;  // (b, s) units
+
+  // ---- tiles per unit and their prefix sums ----
+  for (int u = tid; u < U; u += kThreads) {
+    const int s = u % p.kvp, b = u / p.kvp;
+    int len = p.shard_lens[s * p.B + b];
+    if (len > p.max_pages * kPageTok) {
+      if (blockIdx.x == 0) raise_dev_error(p.err, HELIX_DEVERR_CAPACITY);
+      len = p.max_pages * kPageTok;
+    }
+    pre[u + 1] = len > 0 ? (len + kTok - 1) / kTok : 0;
+  }
+  if (tid == 0) {
+    pre[0] = 0;
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&tail->stage_full[i], 1);
+      mbar_init(&tail->stage_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tail->s_full[i], 1);
+      mbar_init(&tail->s_empty[i], kHeads);
+      mbar_init(&tail->p_full[i], kHeads);
+      mbar_init(&tail->p_empty[i], 1);
+      mbar_init(&tail->x_full[i], kHeads);  // arrivals from the peer's 128 softmax threads
+      mbar_init(&tail->x_free[i], kHeads);
+    }
+    mbar_init(&tail->q_full, 1);
+    mbar_init(&tail->q_empty, 1);
+    tail->flag = 0;
+    tail->abort_ = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {  // allocate all 512 TMEM columns (one CTA per SM)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tail->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (U + 31) / 32;
+    const int lo = 1 + lane * per, hi = min(U + 1, lo + per);
+    int run = 0;
+    for (int i = lo; i < hi; ++i) run += pre[i];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int acc = incl - run;
+    for (int i = lo; i < hi; ++i) {
+      acc += pre[i];
+      pre[i] = acc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
+
+  const uint32_t tmem = tail->tmem_base;
+  const long long W = pre[U];
+  // units with no tokens: O_s = 0, lse_s = -inf (this CTA's value half)
+  for (int u = pair; u < U; u += npairs) {
+    if (pre[u + 1] != pre[u]) continue;
+    const int s = u % p.kvp, b = u / p.kvp;
+    const size_t row0 = ((size_t)s * p.B + b) * kHeads;
+    for (int i = tid; i < kHeads * kHalfDV; i += kThreads)
+      p.o_part[(row0 + i / kHalfDV) * kDV + rank * kHalfDV + i % kHalfDV] = 0.f;
+    if (rank == 0)
+      for (int i = tid; i < kHeads; i += kThreads) p.lse[row0 + i] = -INFINITY;
+  }
+  const int Geff = (int)min((long long)npairs, W);
+  const bool active = pair < Geff;
+  const long long g_begin = active ? range_begin(pair, W, Geff) : 0;
+  const long long g_end = active ? range_begin(pair + 1, W, Geff) : 0;
+  int u_first = 0;
+  if (active) {
+    int lo = 0, hi = U;
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (pre[mid] <= g_begin) lo = mid; else hi = mid;
+    }
+    u_first = lo;
+    while (pre[u_first + 1] <= g_begin) ++u_first;
+  }
+
+  if (warp == 4) {
+    // ===================================== TMA producer ========================================
+    if (lane == 0 && active) {
+      prefetch_tensormap(&tmC);
+      prefetch_tensormap(&tmQ);
+      int u = u_first, cur = -1, qcount = 0;
+      int stage = 0;
+      uint32_t round = 0;
+      for (long long g = g_begin; g < g_end; ++g) {
+        if (*(volatile int*)&tail->abort_) break;
+        while (pre[u + 1] <= g) ++u;
+        const int s = u % p.kvp, b = u / p.kvp;
+        if (u != cur) {  // (re)load this CTA's half of q for request b
+          if (qcount > 0 && !mbar_wait(&tail->q_empty, (qcount - 1) & 1)) {
+            raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
+            *(volatile int*)&tail->abort_ = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->q_full, kQBytes);
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_2d(q_s + c * kHeads * 128, &tmQ, (4 * rank + c) * 64, b * kHeads,
+                        &tail->q_full);
+          cur = u;
+          ++qcount;
+        }
+        if (round > 0 && !mbar_wait(&tail->stage_empty[stage], (round - 1) & 1)) {
+          raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
+          *(volatile int*)&tail->abort_ = 1;
+          break;
+        }
+        const int lt = (int)(g - pre[u]);  // tile within the unit
+        const int page = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + lt / 2);
+        if (page < 0 || page >= p.num_pages) {
+          raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
+          tail->stage_ok[stage] = 0;
+          mbar_arrive(&tail->stage_full[stage]);
+        } else {
+          tail->stage_ok[stage] = 1;
+          mbar_arrive_expect_tx(&tail->stage_full[stage], kStageBytes);
+          uint8_t* st = stage_s + stage * kStageBytes;
+          const int row = page * kPageTok + (lt & 1) * kTok;
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_2d(st + c * kTok * 128, &tmC, (4 * rank + c) * 64, row,
+                        &tail->stage_full[stage]);
+        }
+        if (++stage == kNS) { stage = 0; ++round; }
+      }
+    }
+  } else if (warp == 5) {
+    // ====================================== MMA issuer =========================================
+    if (lane == 0 && active) {
+      constexpr uint32_t idS = make_idesc(128, kTok, false);
+      constexpr uint32_t idPV = make_idesc(128, kHalfDV, true);
+      int u = u_first, cur = -1, qcount = 0;
+      bool dead = false;
+      auto do_pv = [&](long long i, bool fresh) {  // O += P(i) V(i)
+        const int pb = (int)(i & 1);
+        const int st = (int)(i % kNS);
+        if (!mbar_wait(&tail->p_full[pb], (uint32_t)((i >> 1) & 1))) return false;
+        tc_fence_after();
+        const uint32_t pbase = smem_u32(p_s + pb * kPBytes);
+        const uint32_t vbase = smem_u32(stage_s + st * kStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < kTok / 16; ++ks) {
+          // A = P [128 heads x 16 tokens], K-major, 64-byte swizzle, 8-row groups 512 B apart
+          const uint64_t a = smem_desc(pbase + ks * 32, 16, 512, kSwizzle64);
+          // B = V [16 tokens x 256 columns], MN-major, 128-byte swizzle: 64-column groups one
+          // 32-row chunk (4 KiB) apart, 8-token groups 1 KiB apart
+          const uint64_t bdesc = smem_desc(vbase + ks * 16 * 128, kTok * 128, 1024, kSwizzle128);
+          tc_mma(tmem, a, bdesc, idPV, !(fresh && ks == 0));
+        }
+        tc_commit(&tail->stage_empty[st]);
+        tc_commit(&tail->p_empty[pb]);
+        return true;
+      };
+      long long i = 0;
+      bool prev_fresh = false;  // tile i-1 starts a segment (its P V overwrites O)
+      for (long long g = g_begin; g < g_end && !dead; ++g, ++i) {
+        if (*(volatile int*)&tail->abort_) { dead = true; break; }
+        while (pre[u + 1] <= g) ++u;
+        const bool fresh = g == g_begin || g == pre[u];
+        if (u != cur) {
+          if (!mbar_wait(&tail->q_full, qcount & 1)) { dead = true; break; }
+          cur = u;
+          ++qcount;
+        }
+        const int st = (int)(i % kNS);
+        const int sb = (int)(i & 1);
+        if (!mbar_wait(&tail->stage_full[st], (uint32_t)((i / kNS) & 1))) { dead = true; break; }
+        if (i >= 2 && !mbar_wait(&tail->s_empty[sb], (uint32_t)(((i - 2) >> 1) & 1))) {
+          dead = true;
+          break;
+        }
+        tc_fence_after();
+        // S_partial(i) = q[:, half] C_tile[:, half]^T, 18 k-steps of 16 over this CTA's 288 columns
+        const uint32_t qbase = smem_u32(q_s), cbase = smem_u32(stage_s + st * kStageBytes);
+#pragma unroll 1
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          const int e = (int)rank * 32 + ks * 16;  // element offset inside this CTA's 5 chunks
+          const int ch = e >> 6, off = (e & 63) * 2;
+          const uint64_t a = smem_desc(qbase + ch * kHeads * 128 + off, 16, 1024, kSwizzle128);
+          const uint64_t bdesc = smem_desc(cbase + ch * kTok * 128 + off, 16, 1024, kSwizzle128);
+          tc_mma(tmem + kHalfDV + sb * kTok, a, bdesc, idS, ks > 0);
+        }
+        tc_commit(&tail->s_full[sb]);
+        // the last tile of a unit (or of the range) releases q for the next unit
+        if (g + 1 == g_end || g + 1 == pre[u + 1]) tc_commit(&tail->q_empty);
+        if (i >= 1 && !do_pv(i - 1, prev_fresh)) { dead = true; break; }
+        prev_fresh = fresh;
+      }
+      if (!dead && i >= 1) do_pv(i - 1, prev_fresh);
+      if (dead) {
+        raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
+        *(volatile int*)&tail->abort_ = 1;
+      }
+    }
+  } else {
+    // ================================= softmax / epilogue warps ================================
+    const int h = tid;  // head row = TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    float m_use = -INFINITY, l_run = 0.f, lb_run = 0.f;
+    bool has_o = false;  // O holds a partial sum for the current segment
+    bool dead = !active;
+    int u = u_first;
+    long long seg_begin = g_begin;
+    const uint32_t x_peer = map_peer(smem_u32(x_s), peer);
+    const uint32_t xfull_peer = map_peer(smem_u32(&tail->x_full[0]), peer);
+    const uint32_t xfree_peer = map_peer(smem_u32(&tail->x_free[0]), peer);
+    // warp-uniform bounded waits: tcgen05.ld / st below are warp-collective
+    auto wwait = [&](uint64_t* bar, uint32_t parity, bool cluster_scope) {
+      if (dead) return;
+      const bool ok = cluster_scope ? mbar_wait_cluster(bar, parity) : mbar_wait(bar, parity);
+      if (!__all_sync(0xffffffffu, ok)) dead = true;
+    };
+    long long i = 0;
+    for (long long g = g_begin; g < g_end; ++g, ++i) {
+      while (pre[u + 1] <= g) ++u;
+      const int s = u % p.kvp, b = u / p.kvp;
+      const int lt = (int)(g - pre[u]);
+      int len = p.shard_lens[s * p.B + b];
+      const int nvalid = min(kTok, len - lt * kTok);
+      const int sb = (int)(i & 1), xb = (int)(i & 1), pb = (int)(i & 1);
+      const int st_i = (int)(i % kNS);
+      const uint32_t ph = (uint32_t)((i >> 1) & 1);
+      dead = __any_sync(0xffffffffu, dead || *(volatile int*)&tail->abort_ != 0);
+      float sv[32];
+      wwait(&tail->s_full[sb], ph, false);
+      // also observe the tile's load barrier: orders the stage's validity flag and its data before
+      // the zeroing of rows past the end of the history below
+      wwait(&tail->stage_full[st_i], (uint32_t)((i / kNS) & 1), false);
+      const bool tile_ok = tail->stage_ok[st_i] != 0;
+      if (!dead) {
+        tc_fence_after();
+        tmem_ld32(tl + kHalfDV + sb * kTok, sv);
+        tc_fence_before();
+      } else {
+#pragma unroll
+        for (int c = 0; c < kTok; ++c) sv[c] = 0.f;
+      }
+      mbar_arrive(&tail->s_empty[sb]);
+      // ---- swap partial scores with the peer CTA ----
+      if (i >= 2) wwait(&tail->x_free[xb], (uint32_t)(((i - 2) >> 1) & 1), true);
+      {
+        const uint32_t dst = x_peer + (uint32_t)((xb * kHeads + h) * kXStride * 4);
+#pragma unroll
+        for (int c = 0; c < kTok; c += 4) st_cluster_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3]);
+      }
+      remote_arrive(xfull_peer + xb * 8);
+      wwait(&tail->x_full[xb], ph, true);
+      {
+        const float* mine = x_s + (size_t)(xb * kHeads + h) * kXStride;
+#pragma unroll
+        for (int c = 0; c < kTok; c += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(mine + c);
+          sv[c] += v.x;
+          sv[c + 1] += v.y;
+          sv[c + 2] += v.z;
+          sv[c + 3] += v.w;
+        }
+      }
+      remote_arrive(xfree_peer + xb * 8);
+      // ---- online softmax (base 2), lazy rescale ----
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTok; ++c) {
+        sv[c] = (c < nvalid && tile_ok) ? sv[c] * sl2 : -INFINITY;
+        mx = fmaxf(mx, sv[c]);
+      }
+      // V rows past the end of the history are zeroed before the P V product reads them
+      if (nvalid < kTok && !dead) {
+        uint8_t* st = stage_s + (i % kNS) * kStageBytes;
+        for (int e = h; e < (kTok - nvalid) * 4 * 8; e += kHeads) {
+          const int row = nvalid + e / 32, rem = e % 32;
+          *reinterpret_cast<uint4*>(st + (rem / 8) * kTok * 128 + row * 128 + (rem % 8) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      bool rescale = false;
+      float alpha = 1.f;
+      if (!has_o) {
+        if (mx > -INFINITY) m_use = mx;
+      } else if (mx > m_use + 8.f) {
+        alpha = fast_exp2(m_use - mx);
+        m_use = mx;
+        rescale = true;
+      }
+      const float mb = m_use == -INFINITY ? 0.f : m_use;
+      float psum = 0.f, pbsum = 0.f;
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = 0; c < kTok; c += 2) {
+        const float p0 = fast_exp2(sv[c] - mb), p1 = fast_exp2(sv[c + 1] - mb);
+        psum += p0 + p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+        pbsum += bf16_lo_to_f32(pk[c / 2]) + bf16_hi_to_f32(pk[c / 2]);
+      }
+      // P(i) goes into buffer pb, last read by PV(i-2); a rescale also needs PV(i-1) finished
+      if (i >= 2) wwait(&tail->p_empty[pb], (uint32_t)(((i - 2) >> 1) & 1), false);
+      if (__any_sync(0xffffffffu, rescale) && !dead) {
+        if (i >= 1) wwait(&tail->p_empty[pb ^ 1], (uint32_t)(((i - 1) >> 1) & 1), false);
+        tc_fence_after();
+        for (int c = 0; c < kHalfDV; c += 32) {
+          float o[32];
+          tmem_ld32(tl + c, o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(tl + c, o);
+        }
+        tc_fence_before();
+      }
+      if (rescale) {
+        l_run *= alpha;
+        lb_run *= alpha;
+      }
+      l_run += psum;
+      lb_run += pbsum;
+      has_o = true;
+      {  // P row h: 32 bf16 = four 16-byte chunks, 64-byte swizzle (chunk ^= (h >> 1) & 3)
+        uint8_t* prow = p_s + pb * kPBytes + h * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ ((h >> 1) & 3)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&tail->p_full[pb]);
+
+      // ---- end of a segment ----
+      if (g + 1 == g_end || g + 1 == pre[u + 1]) {
+        // O is complete once PV(i) has finished
+        wwait(&tail->p_empty[pb], ph, false);
+        tc_fence_after();
+        const size_t orow = ((size_t)s * p.B + b) * kHeads + h;
+        const bool whole = seg_begin == pre[u] && g + 1 == pre[u + 1];
+        const float M = m_use;
+        float* rec = nullptr;
+        if (!whole) {
+          const int slot = (g_begin >= pre[u]) ? 0 : 1;
+          rec = p.seg + (((size_t)pair * 2 + slot) * 2 + rank) * kRec;
+        }
+        const float inv = lb_run > 0.f ? 1.f / lb_run : 0.f;
+        for (int c = 0; c < kHalfDV; c += 32) {
+          float o[32];
+          if (!dead) tmem_ld32(tl + c, o);
+          else
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = 0.f;
+          float* dst = whole ? p.o_part + orow * kDV + rank * kHalfDV + c : rec + h * kHalfDV + c;
+          const float f = whole ? inv : 1.f;
+#pragma unroll
+          for (int k = 0; k < 32; k += 4)
+            *reinterpret_cast<float4*>(dst + k) =
+                make_float4(o[k] * f, o[k + 1] * f, o[k + 2] * f, o[k + 3] * f);
+        }
+        tc_fence_before();
+        if (whole) {
+          if (rank == 0) p.lse[orow] = l_run > 0.f ? (M + log2f(l_run)) * kLn2 : -INFINITY;
+        } else {
+          rec[kHeads * kHalfDV + h] = M;
+          rec[kHeads * kHalfDV + kHeads + h] = l_run;
+          rec[kHeads * kHalfDV + 2 * kHeads + h] = lb_run;
+          __threadfence();
+          named_barrier_sync(1, kHeads);
+          const int c_lo = cta_of(pre[u], W, Geff), c_hi = cta_of((long long)pre[u + 1] - 1, W, Geff);
+          if (h == 0) {
+            const int ticket = atomicAdd(&p.tickets[u * 2 + rank], 1);
+            tail->flag = ticket == c_hi - c_lo;
+          }
+          named_barrier_sync(1, kHeads);
+          if (tail->flag) {  // merge every cluster's segment of this unit, for this value half
+            __threadfence();
+            float Mm = -INFINITY;
+            for (int c = c_lo; c <= c_hi; ++c) {
+              const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
+              Mm = fmaxf(Mm, __ldcg(p.seg + (((size_t)c * 2 + sl) * 2 + rank) * kRec +
+                                    kHeads * kHalfDV + h));
+            }
+            const float Mmu = Mm == -INFINITY ? 0.f : Mm;
+            float Lm = 0.f, LBm = 0.f;
+            for (int c = c_lo; c <= c_hi; ++c) {
+              const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
+              const float* rc = p.seg + (((size_t)c * 2 + sl) * 2 + rank) * kRec;
+              const float w_ = fast_exp2(__ldcg(rc + kHeads * kHalfDV + h) - Mmu);
+              Lm += __ldcg(rc + kHeads * kHalfDV + kHeads + h) * w_;
+              LBm += __ldcg(rc + kHeads * kHalfDV + 2 * kHeads + h) * w_;
+            }
+            const float invm = LBm > 0.f ? 1.f / LBm : 0.f;
+            for (int cc = 0; cc < kHalfDV; cc += 4) {
+              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int c = c_lo; c <= c_hi; ++c) {
+                const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
+                const float* rc = p.seg + (((size_t)c * 2 + sl) * 2 + rank) * kRec;
+                const float w_ = fast_exp2(__ldcg(rc + kHeads * kHalfDV + h) - Mmu);
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(rc + h * kHalfDV + cc));
+                acc.x += v.x * w_;
+                acc.y += v.y * w_;
+                acc.z += v.z * w_;
+                acc.w += v.w * w_;
+              }
+              *reinterpret_cast<float4*>(p.o_part + orow * kDV + rank * kHalfDV + cc) =
+                  make_float4(acc.x * invm, acc.y * invm, acc.z * invm, acc.w * invm);
+            }
+            if (rank == 0) p.lse[orow] = Lm > 0.f ? (Mm + log2f(Lm)) * kLn2 : -INFINITY;
+            named_barrier_sync(1, kHeads);
+            if (h == 0) p.tickets[u * 2 + rank] = 0;
+          }
+        }
+        named_barrier_sync(1, kHeads);
+        m_use = -INFINITY;
+        l_run = lb_run = 0.f;
+        has_o = false;
+        seg_begin = g + 1;
+      }
+    }
+  }
+
+  // ---- teardown: every thread of both CTAs gets here (all waits above are bounded) ----
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no remote store or arrival can target this CTA after this point
+  if (warp == 5) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace
+
+size_t mla_partial_smem_bytes(int units) { return kSmemFixed + (size_t)(units + 1) * sizeof(int); }
+size_t mla_segment_record_floats() { return kRec; }
+
+helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmQ,
+                                const MlaParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = mla_partial_smem_bytes(p.units);
+  if (cudaFuncSetAttribute(mla_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return HELIX_ERR_CUDA;
+  mla_partial_kernel<<<grid, kThreads, smem, stream>>>(tmC, tmQ, p);
+  return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
+}
+
+}  // namespace helix

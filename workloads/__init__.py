@@ -269,3 +269,8 @@ def append_bytes(w: Workload, n_new: int = 1) -> int:
 
 def step_bytes(w: Workload, lens, n_new: int = 1) -> int:
     return append_bytes(w, n_new) + partial_bytes(w, lens) + combine_bytes(w)
+
+
+def partial_flops(w: Workload, lens) -> float:
+    """Algorithmic flops of the partial attention: 2 * heads * tokens * (K width + V width)."""
+    return 2.0 * w.Hq * sum(lens) * (w.d + w.dv)
