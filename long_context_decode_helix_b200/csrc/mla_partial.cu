@@ -47,10 +47,11 @@ constexpr int kTok = 32;                   // tokens per tile
 constexpr int kPageTok = 64;               // tokens per page
 constexpr int kChunks = 5;                 // 64-column chunks of a latent row per CTA
 constexpr int kKSteps = 18;                // 288 / 16
-constexpr int kNS = 4;                     // tile stages
+constexpr int kNS = 5;                     // tile stages
+constexpr int kNX = 2;                     // score-exchange buffers
 constexpr int kStageBytes = kTok * kChunks * 128;     // 20 KiB
 constexpr int kQBytes = kHeads * kChunks * 128;        // 80 KiB
-constexpr int kPBytes = kHeads * kTok * 2;             // 8 KiB (bf16 P tile, 64-byte rows)
+constexpr uint32_t kSCol = 256, kPCol = 320;           // TMEM columns: O [0,256), S 2x32, P 2x16
 constexpr int kXStride = kTok + 4;                     // padded fp32 row of the exchange buffer
 constexpr int kXBytes = kHeads * kXStride * 4;         // 18 KiB
 constexpr int kThreads = 6 * 32;
@@ -61,7 +62,7 @@ struct MlaTail {
   uint64_t stage_full[kNS], stage_empty[kNS];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
-  uint64_t x_full[2], x_free[2];
+  uint64_t x_full[kNX], x_free[kNX];
   uint64_t q_full, q_empty;
   int stage_ok[kNS];
   uint32_t tmem_base;
@@ -69,7 +70,7 @@ struct MlaTail {
   int abort_;
 };
 
-constexpr size_t kSmemFixed = 1024 + kQBytes + kNS * kStageBytes + 2 * kPBytes + 2 * kXBytes +
+constexpr size_t kSmemFixed = 1024 + kQBytes + kNS * kStageBytes + kNX * kXBytes +
                               sizeof(MlaTail);
 
 // ------------------------------------------------------------------------------------------------
@@ -90,15 +91,28 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t local_addr, uint32_t rank)
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void remote_arrive(uint32_t cluster_bar_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+// Relaxed remote arrival (no implicit cluster-scope fence). Used only to hand a buffer back after
+// reading it; the caller makes the arrival depend on every loaded value first (keep_alive), so the
+// loads have completed before the arrival can be issued.
+__device__ __forceinline__ void remote_arrive_relaxed(uint32_t cluster_bar_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                    cluster_bar_addr)
                : "memory");
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
+template <int N>
+__device__ __forceinline__ void keep_alive(const float (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" ::"f"(v[i]));
+}
+// Asynchronous store into the peer CTA's shared memory; its completion counts `16` bytes against
+// the transaction count of the peer's mbarrier (no fence needed on either side).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d,
+                                            uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(addr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+      : "memory");
 }
 // wait with cluster-scope acquire (data written by the peer CTA)
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
@@ -113,10 +127,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
 }
@@ -131,6 +148,25 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+// D (+)= A B with A read from tensor memory (K-major: row m in lane m, two bf16 per column)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, bool accumulate) {
@@ -205,9 +241,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* q_s = smem;                                   // [5 chunks][128 rows][128 B]
   uint8_t* stage_s = q_s + kQBytes;                      // [kNS][5 chunks][32 rows][128 B]
-  uint8_t* p_s = stage_s + kNS * kStageBytes;            // [2][128 rows][64 B]
-  float* x_s = reinterpret_cast<float*>(p_s + 2 * kPBytes);  // [2][128][kXStride]
-  MlaTail* tail = reinterpret_cast<MlaTail*>(x_s + 2 * kHeads * kXStride);
+  float* x_s = reinterpret_cast<float*>(stage_s + kNS * kStageBytes);  // [kNX][128][kXStride]
+  MlaTail* tail = reinterpret_cast<MlaTail*>(x_s + kNX * kHeads * kXStride);
   int* pre = reinterpret_cast<int*>(tail + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -235,17 +270,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tail->s_full[i], 1);
-      mbar_init(&tail->s_empty[i], kHeads);
-      mbar_init(&tail->p_full[i], kHeads);
+      mbar_init(&tail->s_empty[i], 4);  // one arrival per softmax warp
+      mbar_init(&tail->p_full[i], 4);
       mbar_init(&tail->p_empty[i], 1);
-      mbar_init(&tail->x_full[i], kHeads);  // arrivals from the peer's 128 softmax threads
-      mbar_init(&tail->x_free[i], kHeads);
+    }
+    for (int i = 0; i < kNX; ++i) {
+      // x_full: armed by this CTA with the expected bytes, completed by the peer's async stores
+      mbar_init(&tail->x_full[i], 1);
+      mbar_init(&tail->x_free[i], 4);  // one arrival per softmax warp of the peer CTA
     }
     mbar_init(&tail->q_full, 1);
     mbar_init(&tail->q_empty, 1);
     tail->flag = 0;
     tail->abort_ = 0;
     fence_mbar_init();
+    // arm the exchange barriers for the first kNX tiles (128 rows x 32 fp32 scores each)
+    for (int i = 0; i < kNX; ++i) mbar_arrive_expect_tx(&tail->x_full[i], kHeads * kTok * 4);
   }
   if (warp == 5) {  // allocate all 512 TMEM columns (one CTA per SM)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -355,66 +395,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 5) {
     // ====================================== MMA issuer =========================================
     if (lane == 0 && active) {
+      // Event-driven issue: the next score tile S(ns) goes out as soon as its stage has landed and
+      // its TMEM buffer is free, independent of the P V products, which follow the softmax.
       constexpr uint32_t idS = make_idesc(128, kTok, false);
       constexpr uint32_t idPV = make_idesc(128, kHalfDV, true);
-      int u = u_first, cur = -1, qcount = 0;
+      const long long n = g_end - g_begin;
+      long long ns = 0, npv = 0;
+      int u_s = u_first, u_pv = u_first, cur = -1, qcount = 0;
       bool dead = false;
-      auto do_pv = [&](long long i, bool fresh) {  // O += P(i) V(i)
-        const int pb = (int)(i & 1);
-        const int st = (int)(i % kNS);
-        if (!mbar_wait(&tail->p_full[pb], (uint32_t)((i >> 1) & 1))) return false;
-        tc_fence_after();
-        const uint32_t pbase = smem_u32(p_s + pb * kPBytes);
-        const uint32_t vbase = smem_u32(stage_s + st * kStageBytes);
+      uint64_t t_last = 0;
+      int idle = 0;
+      const uint32_t qbase = smem_u32(q_s);
+      while (npv < n && !dead) {
+        bool progress = false;
+        // P V first: it is on the critical path (it frees the tile's stage and the P buffer)
+        if (npv < ns) {
+          const int pb = (int)(npv & 1);
+          if (mbar_test(&tail->p_full[pb], (uint32_t)((npv >> 1) & 1))) {
+            const long long g = g_begin + npv;
+            while (pre[u_pv + 1] <= g) ++u_pv;
+            const bool fresh = g == g_begin || g == pre[u_pv];  // first tile of a segment
+            const int st = (int)(npv % kNS);
+            tc_fence_after();
+            const uint32_t vbase = smem_u32(stage_s + st * kStageBytes);
 #pragma unroll
-        for (int ks = 0; ks < kTok / 16; ++ks) {
-          // A = P [128 heads x 16 tokens], K-major, 64-byte swizzle, 8-row groups 512 B apart
-          const uint64_t a = smem_desc(pbase + ks * 32, 16, 512, kSwizzle64);
-          // B = V [16 tokens x 256 columns], MN-major, 128-byte swizzle: 64-column groups one
-          // 32-row chunk (4 KiB) apart, 8-token groups 1 KiB apart
-          const uint64_t bdesc = smem_desc(vbase + ks * 16 * 128, kTok * 128, 1024, kSwizzle128);
-          tc_mma(tmem, a, bdesc, idPV, !(fresh && ks == 0));
+            for (int ks = 0; ks < kTok / 16; ++ks) {
+              // A = P [128 heads x 16 tokens] from TMEM (8 columns per 16 tokens)
+              // B = V [16 tokens x 256 columns], MN-major, 128-byte swizzle: 64-column groups one
+              // 32-row chunk (4 KiB) apart, 8-token groups 1 KiB apart
+              const uint64_t bdesc =
+                  smem_desc(vbase + ks * 16 * 128, kTok * 128, 1024, kSwizzle128);
+              tc_mma_ts(tmem, tmem + kPCol + pb * 16 + ks * 8, bdesc, idPV, !(fresh && ks == 0));
+            }
+            tc_commit(&tail->stage_empty[st]);
+            tc_commit(&tail->p_empty[pb]);
+            ++npv;
+            progress = true;
+          }
         }
-        tc_commit(&tail->stage_empty[st]);
-        tc_commit(&tail->p_empty[pb]);
-        return true;
-      };
-      long long i = 0;
-      bool prev_fresh = false;  // tile i-1 starts a segment (its P V overwrites O)
-      for (long long g = g_begin; g < g_end && !dead; ++g, ++i) {
-        if (*(volatile int*)&tail->abort_) { dead = true; break; }
-        while (pre[u + 1] <= g) ++u;
-        const bool fresh = g == g_begin || g == pre[u];
-        if (u != cur) {
-          if (!mbar_wait(&tail->q_full, qcount & 1)) { dead = true; break; }
-          cur = u;
-          ++qcount;
+        if (ns < n) {
+          const long long g = g_begin + ns;
+          while (pre[u_s + 1] <= g) ++u_s;
+          if (u_s != cur && mbar_test(&tail->q_full, qcount & 1)) {  // this unit's q has landed
+            cur = u_s;
+            ++qcount;
+          }
+          const int st = (int)(ns % kNS), sb = (int)(ns & 1);
+          if (u_s == cur && mbar_test(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) &&
+              (ns < 2 || mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - 2) >> 1) & 1)))) {
+            tc_fence_after();
+            // S_partial = q[:, half] C_tile[:, half]^T: 18 k-steps of 16 over this CTA's columns
+            // Descriptors are built once per tile; a k-step only advances the start address
+            // (16-byte units): 32 B inside a 128-byte swizzle row, one chunk (q: 16 KiB, tile:
+            // 4 KiB) per 4 k-steps. This CTA's columns start 32 * rank elements into its chunks.
+            const uint64_t a0 = smem_desc(qbase, 16, 1024, kSwizzle128);
+            const uint64_t b0 = smem_desc(smem_u32(stage_s + st * kStageBytes), 16, 1024,
+                                          kSwizzle128);
+            const uint32_t d_s = tmem + kSCol + sb * kTok;
+#pragma unroll
+            for (int ks = 0; ks < kKSteps; ++ks) {
+              const uint32_t kk = (uint32_t)ks + 2u * rank;  // 16-element step inside the chunks
+              const uint32_t ch = kk >> 2, in_row = (kk & 3u) * 2u;
+              tc_mma(d_s, a0 + ch * (kHeads * 128 / 16) + in_row,
+                     b0 + ch * (kTok * 128 / 16) + in_row, idS, ks > 0);
+            }
+            tc_commit(&tail->s_full[sb]);
+            // the last tile of a unit (or of the range) releases q for the next unit
+            if (g + 1 == g_end || g + 1 == pre[u_s + 1]) tc_commit(&tail->q_empty);
+            ++ns;
+            progress = true;
+          }
         }
-        const int st = (int)(i % kNS);
-        const int sb = (int)(i & 1);
-        if (!mbar_wait(&tail->stage_full[st], (uint32_t)((i / kNS) & 1))) { dead = true; break; }
-        if (i >= 2 && !mbar_wait(&tail->s_empty[sb], (uint32_t)(((i - 2) >> 1) & 1))) {
-          dead = true;
-          break;
+        // bounded: give up after the wait limit passes without any progress (t_last = 0 means the
+        // clock is not running; it starts on the first batch of 256 idle polls)
+        if (progress) {
+          idle = 0;
+          t_last = 0;
+        } else if (++idle >= 256) {
+          idle = 0;
+          if (*(volatile int*)&tail->abort_) dead = true;
+          const uint64_t now = global_timer_ns();
+          if (t_last == 0) t_last = now;
+          else if (now - t_last > kWaitLimitNs) dead = true;
         }
-        tc_fence_after();
-        // S_partial(i) = q[:, half] C_tile[:, half]^T, 18 k-steps of 16 over this CTA's 288 columns
-        const uint32_t qbase = smem_u32(q_s), cbase = smem_u32(stage_s + st * kStageBytes);
-#pragma unroll 1
-        for (int ks = 0; ks < kKSteps; ++ks) {
-          const int e = (int)rank * 32 + ks * 16;  // element offset inside this CTA's 5 chunks
-          const int ch = e >> 6, off = (e & 63) * 2;
-          const uint64_t a = smem_desc(qbase + ch * kHeads * 128 + off, 16, 1024, kSwizzle128);
-          const uint64_t bdesc = smem_desc(cbase + ch * kTok * 128 + off, 16, 1024, kSwizzle128);
-          tc_mma(tmem + kHalfDV + sb * kTok, a, bdesc, idS, ks > 0);
-        }
-        tc_commit(&tail->s_full[sb]);
-        // the last tile of a unit (or of the range) releases q for the next unit
-        if (g + 1 == g_end || g + 1 == pre[u + 1]) tc_commit(&tail->q_empty);
-        if (i >= 1 && !do_pv(i - 1, prev_fresh)) { dead = true; break; }
-        prev_fresh = fresh;
       }
-      if (!dead && i >= 1) do_pv(i - 1, prev_fresh);
       if (dead) {
         raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
         *(volatile int*)&tail->abort_ = 1;
@@ -439,41 +503,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool ok = cluster_scope ? mbar_wait_cluster(bar, parity) : mbar_wait(bar, parity);
       if (!__all_sync(0xffffffffu, ok)) dead = true;
     };
-    long long i = 0;
-    for (long long g = g_begin; g < g_end; ++g, ++i) {
-      while (pre[u + 1] <= g) ++u;
-      const int s = u % p.kvp, b = u / p.kvp;
-      const int lt = (int)(g - pre[u]);
-      int len = p.shard_lens[s * p.B + b];
-      const int nvalid = min(kTok, len - lt * kTok);
-      const int sb = (int)(i & 1), xb = (int)(i & 1), pb = (int)(i & 1);
-      const int st_i = (int)(i % kNS);
-      const uint32_t ph = (uint32_t)((i >> 1) & 1);
+    // Phase A(j): read tile j's partial scores from TMEM and send them to the peer.
+    // Phase B(i): receive the peer's partial for tile i, finish the softmax, hand P to the MMA.
+    // The loop runs A(i+1) before B(i), so the exchange of tile i overlaps the work on tile i+1.
+    auto phase_a = [&](long long j, float (&sv)[32], bool& tile_ok) {
+      const int sb = (int)(j & 1), xb = (int)(j % kNX);
+      const int st_j = (int)(j % kNS);
       dead = __any_sync(0xffffffffu, dead || *(volatile int*)&tail->abort_ != 0);
-      float sv[32];
-      wwait(&tail->s_full[sb], ph, false);
+      wwait(&tail->s_full[sb], (uint32_t)((j >> 1) & 1), false);
       // also observe the tile's load barrier: orders the stage's validity flag and its data before
-      // the zeroing of rows past the end of the history below
-      wwait(&tail->stage_full[st_i], (uint32_t)((i / kNS) & 1), false);
-      const bool tile_ok = tail->stage_ok[st_i] != 0;
+      // the zeroing of rows past the end of the history in phase B
+      wwait(&tail->stage_full[st_j], (uint32_t)((j / kNS) & 1), false);
+      tile_ok = tail->stage_ok[st_j] != 0;
       if (!dead) {
         tc_fence_after();
-        tmem_ld32(tl + kHalfDV + sb * kTok, sv);
+        tmem_ld32(tl + kSCol + sb * kTok, sv);
         tc_fence_before();
       } else {
 #pragma unroll
         for (int c = 0; c < kTok; ++c) sv[c] = 0.f;
       }
-      mbar_arrive(&tail->s_empty[sb]);
-      // ---- swap partial scores with the peer CTA ----
-      if (i >= 2) wwait(&tail->x_free[xb], (uint32_t)(((i - 2) >> 1) & 1), true);
-      {
-        const uint32_t dst = x_peer + (uint32_t)((xb * kHeads + h) * kXStride * 4);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->s_empty[sb]);
+      if (j >= kNX) wwait(&tail->x_free[xb], (uint32_t)(((j - kNX) / kNX) & 1), true);
+      const uint32_t dst = x_peer + (uint32_t)((xb * kHeads + h) * kXStride * 4);
 #pragma unroll
-        for (int c = 0; c < kTok; c += 4) st_cluster_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3]);
-      }
-      remote_arrive(xfull_peer + xb * 8);
-      wwait(&tail->x_full[xb], ph, true);
+      for (int c = 0; c < kTok; c += 4)
+        st_async_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3], xfull_peer + xb * 8);
+    };
+    long long i = 0;
+    auto phase_b = [&](float (&sv)[32], bool tile_ok) -> bool {  // returns true at a segment end
+      const long long g = g_begin + i;
+      while (pre[u + 1] <= g) ++u;
+      const int s = u % p.kvp, b = u / p.kvp;
+      const int lt = (int)(g - pre[u]);
+      const int len = p.shard_lens[s * p.B + b];
+      const int nvalid = min(kTok, len - lt * kTok);
+      const int xb = (int)(i % kNX), pb = (int)(i & 1);
+      wwait(&tail->x_full[xb], (uint32_t)((i / kNX) & 1), true);
       {
         const float* mine = x_s + (size_t)(xb * kHeads + h) * kXStride;
 #pragma unroll
@@ -485,13 +552,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           sv[c + 3] += v.w;
         }
       }
-      remote_arrive(xfree_peer + xb * 8);
+      // re-arm this buffer's barrier for tile i+2 (once every thread here has observed tile i's
+      // phase, which the wait above guarantees for this thread), then release the buffer
+      if (h == 0 && i + kNX < g_end - g_begin)
+        mbar_arrive_expect_tx(&tail->x_full[xb], kHeads * kTok * 4);
+      keep_alive(sv);  // the buffer's loads have returned before the buffer is handed back
+      __syncwarp();
+      if (lane == 0) remote_arrive_relaxed(xfree_peer + xb * 8);
       // ---- online softmax (base 2), lazy rescale ----
-      float mx = -INFINITY;
+      if (nvalid == kTok && tile_ok) {
 #pragma unroll
-      for (int c = 0; c < kTok; ++c) {
-        sv[c] = (c < nvalid && tile_ok) ? sv[c] * sl2 : -INFINITY;
-        mx = fmaxf(mx, sv[c]);
+        for (int c = 0; c < kTok; ++c) sv[c] *= sl2;
+      } else {
+#pragma unroll
+        for (int c = 0; c < kTok; ++c) sv[c] = (c < nvalid && tile_ok) ? sv[c] * sl2 : -INFINITY;
+      }
+      float mx;
+      {  // tree reduction of the row maximum
+        float t[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) t[c] = fmaxf(sv[c], sv[c + 16]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) t[c] = fmaxf(t[c], t[c + 8]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) t[c] = fmaxf(t[c], t[c + 4]);
+        mx = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
       }
       // V rows past the end of the history are zeroed before the P V product reads them
       if (nvalid < kTok && !dead) {
@@ -513,15 +598,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         rescale = true;
       }
       const float mb = m_use == -INFINITY ? 0.f : m_use;
-      float psum = 0.f, pbsum = 0.f;
       uint32_t pk[16];
+      float ps[16];
 #pragma unroll
       for (int c = 0; c < kTok; c += 2) {
         const float p0 = fast_exp2(sv[c] - mb), p1 = fast_exp2(sv[c + 1] - mb);
-        psum += p0 + p1;
+        ps[c / 2] = p0 + p1;
         pk[c / 2] = pack_bf16x2(p0, p1);
-        pbsum += bf16_lo_to_f32(pk[c / 2]) + bf16_hi_to_f32(pk[c / 2]);
       }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) ps[c] += ps[c + 8];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
+      // O is normalised by the fp32 sum (the bf16-rounded weights differ from it by < 2^-9)
+      const float psum = (ps[0] + ps[2]) + (ps[1] + ps[3]);
+      const float pbsum = psum;
       // P(i) goes into buffer pb, last read by PV(i-2); a rescale also needs PV(i-1) finished
       if (i >= 2) wwait(&tail->p_empty[pb], (uint32_t)(((i - 2) >> 1) & 1), false);
       if (__any_sync(0xffffffffu, rescale) && !dead) {
@@ -543,19 +634,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       l_run += psum;
       lb_run += pbsum;
       has_o = true;
-      {  // P row h: 32 bf16 = four 16-byte chunks, 64-byte swizzle (chunk ^= (h >> 1) & 3)
-        uint8_t* prow = p_s + pb * kPBytes + h * 64;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ ((h >> 1) & 3)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
+      // P row h (32 bf16) into this thread's TMEM lane: the A operand of the P V product
+      if (!dead) tmem_st16(tl + kPCol + pb * 16, pk);
       tc_fence_before();
-      mbar_arrive(&tail->p_full[pb]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->p_full[pb]);
+      return g + 1 == g_end || g + 1 == pre[u + 1];
+    };
+    const long long n_tiles = g_end - g_begin;
+    float sv0[32], sv1[32];
+    bool ok0 = false, ok1 = false;
+    if (n_tiles > 0) phase_a(0, sv0, ok0);
+    for (i = 0; i < n_tiles; ++i) {
+      bool seg_end;
+      if ((i & 1) == 0) {
+        if (i + 1 < n_tiles) phase_a(i + 1, sv1, ok1);
+        seg_end = phase_b(sv0, ok0);
+      } else {
+        if (i + 1 < n_tiles) phase_a(i + 1, sv0, ok0);
+        seg_end = phase_b(sv1, ok1);
+      }
+      const long long g = g_begin + i;
+      const int s = u % p.kvp, b = u / p.kvp;
+      const int pb = (int)(i & 1);
+      const uint32_t ph = (uint32_t)((i >> 1) & 1);
 
       // ---- end of a segment ----
-      if (g + 1 == g_end || g + 1 == pre[u + 1]) {
+      if (seg_end) {
         // O is complete once PV(i) has finished
         wwait(&tail->p_empty[pb], ph, false);
         tc_fence_after();
