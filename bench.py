@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--impl", default="helix", choices=["helix", "reference"])
     ap.add_argument("--workload", default="gqa_s1m", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--hopb-groups", type=int, default=4,
+                    help="request groups of the two-stream HOP-B analogue, timed after the main "
+                         "steps and reported under 'hopb' (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=1 << 19,
                     help="history tokens per sampled head group for the CPU oracle")
@@ -268,7 +271,7 @@ def run_helix(args):
     lens = wl.seq_lens(w)
     dev = torch.device("cuda", local)
     K, W = args.steps, args.warmup
-    n_steps = K + W + (K if not args.no_e2e else 0)
+    n_steps = K + W + (K if not args.no_e2e else 0) + (W + K if args.hopb_groups > 0 else 0)
     S_cap = max(lens) + n_steps + 16
 
     # --- state resident in HBM: the history (S_b - 1 tokens), then one new token per step ---
@@ -365,9 +368,43 @@ def run_helix(args):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
+        si += K
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, world)
         e2e = {"value": e2e_ms * 1e3, "unit": "us/step", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
+
+    # --- HOP-B analogue: the combine of request group g on a second stream overlaps the partial of
+    # group g+1; same append, same inputs, timed like the main steps ---
+    hopb = None
+    if args.hopb_groups > 0:
+        ov = hx.Overlap(args.hopb_groups, dev)
+
+        def hopb_step(i):
+            a = {k: v[i] for k, v in step_rows.items()}
+            hx.append(cache, a["k_new"], a.get("v_new"), a.get("k_scale"), a.get("v_scale"))
+            hx.overlapped(cache, q, w.softmax_scale, ov, o_part, lse_part, out, lse_out,
+                          workspace=ws)
+
+        for _ in range(W):
+            hopb_step(si)
+            si += 1
+        barrier(world)
+        torch.cuda.synchronize()
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for i in range(K):
+            hopb_step(si + i)
+        h1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        si += K
+        hopb_ms = max_over_ranks(h0.elapsed_time(h1) / K, world)
+        n_groups = min(args.hopb_groups, w.B)
+        per = -(-w.B // n_groups)
+        hopb = {"groups": -(-w.B // per), "us_per_step": hopb_ms * 1e3,
+                "serial_us_per_step": ms_step * 1e3, "speedup": ms_step / hopb_ms,
+                "gpu_launches": K * (1 + 2 * (-(-w.B // per)))}
+        assert cache.err_bits() == 0, "a HOP-B step reported a device error"
 
     if rank == 0:
         step_bytes = float(np.mean([wl.step_bytes(w, L) for L in lens_at]))
@@ -402,6 +439,7 @@ def run_helix(args):
             "roofline": roof,
             "e2e": e2e,
             "clocks": clk,
+            "hopb": hopb,
         }
         if not args.no_cpu_baseline and world == 1:
             v, desc, cores, _ = cpu_oracle_sample(w, args.cpu_sample_tokens, args.cpu_sample_groups)

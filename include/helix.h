@@ -40,6 +40,7 @@ extern "C" {
 
 /* Same object as cudaStream_t; declared opaquely so this header needs no CUDA headers. */
 typedef struct CUstream_st* helix_stream_t;
+typedef struct CUevent_st* helix_event_t; /* a cudaEvent_t */
 
 typedef enum {
   HELIX_OK = 0,
@@ -165,6 +166,45 @@ helix_status helix_attn_partial(const helix_kv_cache* cache, const void* q, int3
 helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads, int32_t v_dim,
                                 const float* o_partial, const float* lse, void* o_out,
                                 int32_t o_dtype, float* lse_out, helix_stream_t stream);
+
+/*
+ * helix_attn_partial restricted to the requests [b_begin, b_end) (0 <= b_begin <= b_end <= batch).
+ * q, o_partial and lse keep their full shapes and indexing; rows of other requests are neither read
+ * nor written. Same workspace as helix_attn_partial: calls sharing a workspace must be ordered on
+ * the GPU (one stream, or events). b_begin == b_end launches nothing.
+ */
+helix_status helix_attn_partial_range(const helix_kv_cache* cache, const void* q,
+                                      int32_t num_q_heads, float softmax_scale, int32_t b_begin,
+                                      int32_t b_end, float* o_partial, float* lse, void* workspace,
+                                      size_t workspace_bytes, helix_stream_t stream);
+
+/* helix_attn_combine restricted to the requests [b_begin, b_end); full-shape arrays as above. */
+helix_status helix_attn_combine_range(int32_t kvp, int32_t batch, int32_t num_q_heads,
+                                      int32_t v_dim, int32_t b_begin, int32_t b_end,
+                                      const float* o_partial, const float* lse, void* o_out,
+                                      int32_t o_dtype, float* lse_out, helix_stream_t stream);
+
+/*
+ * One-GPU analogue of HOP-B, the batch-wise overlap of one request's exchange with the next
+ * request's attention (ifai.io news, "Decoupling attention and FFN"; NVIDIA blog, Korean edition,
+ * Figure 3). The batch is cut into n_groups contiguous request groups (ceil(B / n_groups) requests
+ * each; n_groups is clamped to B). On stream_a the partial attention of group g runs after that of
+ * group g-1 (they share the workspace); on stream_b the combine of group g waits for it (event
+ * events[g]) and then overlaps the partial of group g+1. Finally stream_a waits for stream_b
+ * (events[n_groups]), so the results are ready when stream_a's work is.
+ *   events : n_groups + 1 CUDA events created by the caller (timing disabled is best)
+ *   other arguments as helix_attn_partial + helix_attn_combine (o_dtype 0 bf16, 1 fp32;
+ *   lse_out may be NULL). stream_a and stream_b must differ.
+ * Results equal helix_attn_partial_range over each group followed by the combine: per request, the
+ * same numbers up to the rounding of how the kernel splits a group's units across CTAs.
+ * Every argument is validated before the first launch.
+ */
+helix_status helix_attn_overlapped(const helix_kv_cache* cache, const void* q, int32_t num_q_heads,
+                                   float softmax_scale, int32_t n_groups, float* o_partial,
+                                   float* lse, void* o_out, int32_t o_dtype, float* lse_out,
+                                   void* workspace, size_t workspace_bytes,
+                                   helix_stream_t stream_a, helix_stream_t stream_b,
+                                   const helix_event_t* events);
 
 /*
  * helix_attn_partial for callers that cannot allocate device memory. The paper has no counterpart;

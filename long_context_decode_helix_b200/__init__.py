@@ -64,6 +64,13 @@ def _load():
     lib.helix_attn_partial_noalloc.restype = I32
     lib.helix_attn_combine.argtypes = [I32, I32, I32, I32, P, P, P, I32, P, P]
     lib.helix_attn_combine.restype = I32
+    lib.helix_attn_partial_range.argtypes = [cache_p, P, I32, F32, I32, I32, P, P, P, SZ, P]
+    lib.helix_attn_partial_range.restype = I32
+    lib.helix_attn_combine_range.argtypes = [I32, I32, I32, I32, I32, I32, P, P, P, I32, P, P]
+    lib.helix_attn_combine_range.restype = I32
+    lib.helix_attn_overlapped.argtypes = [cache_p, P, I32, F32, I32, P, P, P, I32, P, P, SZ, P, P,
+                                          ctypes.POINTER(P)]
+    lib.helix_attn_overlapped.restype = I32
     lib.helix_status_string.argtypes = [I32]
     lib.helix_status_string.restype = ctypes.c_char_p
     lib.helix_version.argtypes = []
@@ -221,6 +228,74 @@ def combine(o_partial: torch.Tensor, lse: torch.Tensor, out=None, lse_out=None,
     o_dtype = 0 if out.dtype == torch.bfloat16 else 1
     _check(lib.helix_attn_combine(P, B, Hq, dv, _ptr(o_partial), _ptr(lse), _ptr(out), o_dtype,
                                   _ptr(lse_out), _stream(stream)), "helix_attn_combine")
+    return out, lse_out
+
+
+def partial_range(cache: KVCache, q: torch.Tensor, softmax_scale: float, b_begin: int, b_end: int,
+                  o_partial: torch.Tensor, lse: torch.Tensor, workspace=None, stream=None):
+    """``helix_attn_partial_range``: partial attention of requests [b_begin, b_end) only, written
+    into the full-shape ``o_partial`` / ``lse``."""
+    B, Hq, _ = q.shape
+    if workspace is None:
+        workspace = cache.workspace(Hq)
+    _check(lib.helix_attn_partial_range(ctypes.byref(cache.struct), _ptr(q), Hq,
+                                        float(softmax_scale), b_begin, b_end, _ptr(o_partial),
+                                        _ptr(lse), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "helix_attn_partial_range")
+    return o_partial, lse
+
+
+def combine_range(o_partial: torch.Tensor, lse: torch.Tensor, b_begin: int, b_end: int, out,
+                  lse_out=None, stream=None):
+    """``helix_attn_combine_range``: combine of requests [b_begin, b_end) into the full-shape
+    ``out`` / ``lse_out``."""
+    P, B, Hq, dv = o_partial.shape
+    o_dtype = 0 if out.dtype == torch.bfloat16 else 1
+    _check(lib.helix_attn_combine_range(P, B, Hq, dv, b_begin, b_end, _ptr(o_partial), _ptr(lse),
+                                        _ptr(out), o_dtype, _ptr(lse_out), _stream(stream)),
+           "helix_attn_combine_range")
+    return out, lse_out
+
+
+class Overlap:
+    """The second stream and the events ``helix_attn_overlapped`` needs, created once."""
+
+    def __init__(self, n_groups: int, device=None):
+        self.n_groups = int(n_groups)
+        self.stream_b = torch.cuda.Stream(device=device)
+        cur = torch.cuda.current_stream(device)
+        self.events = [torch.cuda.Event() for _ in range(self.n_groups + 1)]
+        for e in self.events:  # torch creates the CUDA event lazily, on its first record
+            e.record(cur)
+        self._handles = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
+
+
+def overlapped(cache: KVCache, q: torch.Tensor, softmax_scale: float, overlap: Overlap,
+               o_partial=None, lse=None, out=None, lse_out=None, out_dtype=torch.bfloat16,
+               workspace=None, stream=None):
+    """HOP-B analogue (``helix_attn_overlapped``): per request group, partial attention on
+    ``stream`` and the combine on ``overlap.stream_b``, overlapping the next group's partial.
+    Returns (O, LSE)."""
+    B, Hq, _ = q.shape
+    dev = q.device
+    if o_partial is None:
+        o_partial = torch.empty(cache.kvp, B, Hq, cache.v_dim, dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty(cache.kvp, B, Hq, dtype=torch.float32, device=dev)
+    if out is None:
+        out = torch.empty(B, Hq, cache.v_dim, dtype=out_dtype, device=dev)
+    if lse_out is None:
+        lse_out = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = cache.workspace(Hq)
+    o_dtype = 0 if out.dtype == torch.bfloat16 else 1
+    _check(lib.helix_attn_overlapped(ctypes.byref(cache.struct), _ptr(q), Hq, float(softmax_scale),
+                                     overlap.n_groups, _ptr(o_partial), _ptr(lse), _ptr(out),
+                                     o_dtype, _ptr(lse_out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(stream), _stream(overlap.stream_b),
+                                     overlap._handles), "helix_attn_overlapped")
     return out, lse_out
 
 

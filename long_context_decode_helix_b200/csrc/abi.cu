@@ -141,11 +141,14 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
   int sms = 0, max_smem = 0;
   if (device_sm_count(&sms) != 0 || device_max_smem(&max_smem) != 0) return HELIX_ERR_CUDA;
   plan->units = c->batch * c->num_kv_heads * c->kvp;
-  if (gqa_partial_smem_bytes(c->head_dim, nvfp4, plan->units) > (size_t)max_smem)
-    return HELIX_ERR_CAPACITY;
+  const size_t smem = nvfp4 ? gqa_nvfp4_smem_bytes(plan->units)
+                            : gqa_partial_smem_bytes(c->head_dim, plan->units);
+  if (smem > (size_t)max_smem) return HELIX_ERR_CAPACITY;
   plan->grid = sms;
   plan->ticket_bytes = (((size_t)plan->units * sizeof(int32_t)) + 255) & ~size_t(255);
-  plan->seg_bytes = (size_t)plan->grid * 2 * gqa_segment_record_floats(c->head_dim) * sizeof(float);
+  const size_t rec = nvfp4 ? gqa_nvfp4_segment_record_floats()
+                           : gqa_segment_record_floats(c->head_dim);
+  plan->seg_bytes = (size_t)plan->grid * 2 * rec * sizeof(float);
   return HELIX_OK;
 }
 
@@ -227,9 +230,12 @@ helix_status helix_attn_workspace_size(const helix_kv_cache* c, int32_t num_q_he
   return HELIX_OK;
 }
 
-helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
-                                float softmax_scale, float* o_partial, float* lse, void* workspace,
-                                size_t workspace_bytes, helix_stream_t stream) {
+helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
+                                      int32_t num_q_heads, float softmax_scale, int32_t b_begin,
+                                      int32_t b_end, float* o_partial, float* lse, void* workspace,
+                                      size_t workspace_bytes, helix_stream_t stream) {
+  if (c == nullptr || b_begin < 0 || b_end < b_begin || b_end > c->batch)
+    return HELIX_ERR_INVALID_ARG;
   PartialPlan plan;
   helix_status st = plan_partial(c, num_q_heads, &plan);
   if (st != HELIX_OK) return st;
@@ -239,6 +245,11 @@ helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t 
     return HELIX_ERR_INVALID_ARG;
   if (workspace_bytes < plan.ticket_bytes + plan.seg_bytes) return HELIX_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return HELIX_ERR_INVALID_ARG;
+  if (b_end == b_begin) return HELIX_OK;
+  // units are ordered request-major, so a request range is a contiguous unit range
+  const int units_per_request = plan.units / c->batch;
+  const int u0 = b_begin * units_per_request;
+  const int units = (b_end - b_begin) * units_per_request;
 
   if (c->kind == HELIX_ATTN_MLA) {
     MlaParams m{};
@@ -253,7 +264,8 @@ helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t 
     m.kvp = c->kvp;
     m.max_pages = c->max_pages_per_shard;
     m.num_pages = c->num_pages;
-    m.units = plan.units;
+    m.units = units;
+    m.u0 = u0;
     m.scale_log2 = softmax_scale * 1.4426950408889634f;
     // latent pool as [pages * 64 rows][576], boxes of 64 columns x 32 rows; q as [B * 128][576],
     // boxes of 64 columns x 128 rows; 128-byte swizzle for the tensor-core operand layout
@@ -283,7 +295,8 @@ helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t 
   p.kvp = c->kvp;
   p.max_pages = c->max_pages_per_shard;
   p.num_pages = c->num_pages;
-  p.units = plan.units;
+  p.units = units;
+  p.u0 = u0;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   if (c->kv_dtype == HELIX_KV_NVFP4) {
     p.k_codes = reinterpret_cast<const uint8_t*>(c->k_pool);
@@ -303,17 +316,79 @@ helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t 
   return gqa_partial_bf16_launch(tmK, tmV, p, plan.grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
-helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads, int32_t v_dim,
-                                const float* o_partial, const float* lse, void* o_out,
-                                int32_t o_dtype, float* lse_out, helix_stream_t stream) {
+helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                                float softmax_scale, float* o_partial, float* lse, void* workspace,
+                                size_t workspace_bytes, helix_stream_t stream) {
+  if (c == nullptr) return HELIX_ERR_INVALID_ARG;
+  return helix_attn_partial_range(c, q, num_q_heads, softmax_scale, 0, c->batch, o_partial, lse,
+                                  workspace, workspace_bytes, stream);
+}
+
+helix_status helix_attn_combine_range(int32_t kvp, int32_t batch, int32_t num_q_heads,
+                                      int32_t v_dim, int32_t b_begin, int32_t b_end,
+                                      const float* o_partial, const float* lse, void* o_out,
+                                      int32_t o_dtype, float* lse_out, helix_stream_t stream) {
   if (kvp < 1 || batch < 0 || num_q_heads < 0 || v_dim < 4 || v_dim % 4 != 0)
     return HELIX_ERR_INVALID_ARG;
+  if (b_begin < 0 || b_end < b_begin || b_end > batch) return HELIX_ERR_INVALID_ARG;
   if (o_dtype != 0 && o_dtype != 1) return HELIX_ERR_INVALID_ARG;
   if (o_partial == nullptr || lse == nullptr || o_out == nullptr) return HELIX_ERR_INVALID_ARG;
   if (!aligned16(o_partial) || !aligned4(lse) || !aligned16(o_out) || !aligned4(lse_out))
     return HELIX_ERR_INVALID_ARG;
-  return combine_launch(kvp, batch, num_q_heads, v_dim, o_partial, lse, o_out, o_dtype, lse_out,
-                        reinterpret_cast<cudaStream_t>(stream));
+  return combine_launch(kvp, batch * num_q_heads, b_begin * num_q_heads,
+                        (b_end - b_begin) * num_q_heads, v_dim, o_partial, lse, o_out, o_dtype,
+                        lse_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads, int32_t v_dim,
+                                const float* o_partial, const float* lse, void* o_out,
+                                int32_t o_dtype, float* lse_out, helix_stream_t stream) {
+  return helix_attn_combine_range(kvp, batch, num_q_heads, v_dim, 0, batch, o_partial, lse, o_out,
+                                  o_dtype, lse_out, stream);
+}
+
+helix_status helix_attn_overlapped(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                                   float softmax_scale, int32_t n_groups, float* o_partial,
+                                   float* lse, void* o_out, int32_t o_dtype, float* lse_out,
+                                   void* workspace, size_t workspace_bytes,
+                                   helix_stream_t stream_a, helix_stream_t stream_b,
+                                   const helix_event_t* events) {
+  if (c == nullptr || events == nullptr || n_groups < 1) return HELIX_ERR_INVALID_ARG;
+  if (stream_a == stream_b) return HELIX_ERR_INVALID_ARG;
+  for (int g = 0; g <= n_groups; ++g)
+    if (events[g] == nullptr) return HELIX_ERR_INVALID_ARG;
+  // validate everything before the first launch, so an error launches nothing
+  PartialPlan plan;
+  helix_status st = plan_partial(c, num_q_heads, &plan);
+  if (st != HELIX_OK) return st;
+  if (q == nullptr || o_partial == nullptr || lse == nullptr || workspace == nullptr ||
+      o_out == nullptr || (o_dtype != 0 && o_dtype != 1) || c->v_dim % 4 != 0)
+    return HELIX_ERR_INVALID_ARG;
+  if (!aligned16(o_out) || !aligned4(lse_out)) return HELIX_ERR_INVALID_ARG;
+  const int B = c->batch;
+  const int groups = n_groups < B ? n_groups : B;
+  const int per = (B + groups - 1) / groups;
+  auto sa = reinterpret_cast<cudaStream_t>(stream_a);
+  auto sb = reinterpret_cast<cudaStream_t>(stream_b);
+  for (int g = 0; g * per < B; ++g) {
+    const int b0 = g * per, b1 = b0 + per < B ? b0 + per : B;
+    // stream A: partial attention of request group g (groups run back to back on A, sharing the
+    // workspace); stream B: combine of group g once its partials exist, overlapping group g+1
+    st = helix_attn_partial_range(c, q, num_q_heads, softmax_scale, b0, b1, o_partial, lse,
+                                  workspace, workspace_bytes, stream_a);
+    if (st != HELIX_OK) return st;
+    auto ev = reinterpret_cast<cudaEvent_t>(events[g]);
+    if (cudaEventRecord(ev, sa) != cudaSuccess || cudaStreamWaitEvent(sb, ev, 0) != cudaSuccess)
+      return HELIX_ERR_CUDA;
+    st = helix_attn_combine_range(c->kvp, B, num_q_heads, c->v_dim, b0, b1, o_partial, lse, o_out,
+                                  o_dtype, lse_out, stream_b);
+    if (st != HELIX_OK) return st;
+  }
+  // join: stream A waits for the last combine, so the caller needs to order only against A
+  auto done = reinterpret_cast<cudaEvent_t>(events[n_groups]);
+  if (cudaEventRecord(done, sb) != cudaSuccess || cudaStreamWaitEvent(sa, done, 0) != cudaSuccess)
+    return HELIX_ERR_CUDA;
+  return HELIX_OK;
 }
 
 }  // extern "C"

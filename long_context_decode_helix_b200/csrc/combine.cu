@@ -21,12 +21,13 @@ constexpr int kCombineThreads = 256;
 
 template <bool BF16_OUT>
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(int kvp, int rows, int v_dim, const float* __restrict__ o_part,
-                   const float* __restrict__ lse, void* __restrict__ o_out,
-                   float* __restrict__ lse_out) {
-  const int warp = (blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
+    combine_kernel(int kvp, int rows, int row0, int nrows, int v_dim,
+                   const float* __restrict__ o_part, const float* __restrict__ lse,
+                   void* __restrict__ o_out, float* __restrict__ lse_out) {
+  const int wl = (blockIdx.x * kCombineThreads + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
+  if (wl >= nrows) return;
+  const int warp = row0 + wl;  // (b, h) row of this warp; rows = B * Hq is the shard stride
   float M = -INFINITY;
   for (int s = 0; s < kvp; ++s) M = fmaxf(M, __ldg(lse + (size_t)s * rows + warp));
   const float Mu = M == -INFINITY ? 0.f : M;
@@ -65,18 +66,17 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 }  // namespace
 
-helix_status combine_launch(int kvp, int batch, int num_q_heads, int v_dim, const float* o_partial,
-                            const float* lse, void* o_out, int o_dtype, float* lse_out,
-                            cudaStream_t stream) {
-  const int rows = batch * num_q_heads;
-  if (rows == 0) return HELIX_OK;
-  const int blocks = (rows * 32 + kCombineThreads - 1) / kCombineThreads;
+helix_status combine_launch(int kvp, int rows, int row0, int nrows, int v_dim,
+                            const float* o_partial, const float* lse, void* o_out, int o_dtype,
+                            float* lse_out, cudaStream_t stream) {
+  if (nrows == 0) return HELIX_OK;
+  const int blocks = (nrows * 32 + kCombineThreads - 1) / kCombineThreads;
   if (o_dtype == 0)
-    combine_kernel<true><<<blocks, kCombineThreads, 0, stream>>>(kvp, rows, v_dim, o_partial, lse,
-                                                                 o_out, lse_out);
+    combine_kernel<true><<<blocks, kCombineThreads, 0, stream>>>(kvp, rows, row0, nrows, v_dim,
+                                                                 o_partial, lse, o_out, lse_out);
   else
-    combine_kernel<false><<<blocks, kCombineThreads, 0, stream>>>(kvp, rows, v_dim, o_partial,
-                                                                  lse, o_out, lse_out);
+    combine_kernel<false><<<blocks, kCombineThreads, 0, stream>>>(kvp, rows, row0, nrows, v_dim,
+                                                                  o_partial, lse, o_out, lse_out);
   return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
 }
 

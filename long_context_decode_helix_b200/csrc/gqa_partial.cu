@@ -1,4 +1,5 @@
-// gqa_partial.cu -- per-shard partial decode attention for grouped-query attention (bf16 or NVFP4 KV).
+// gqa_partial.cu -- per-shard partial decode attention for grouped-query attention over a bf16 KV
+// cache (the NVFP4 cache has its own kernel, gqa_partial_nvfp4.cu).
 //
 // What it computes (paper summary "Helix Parallelism: Rethinking Sharding Strategies for
 // Interactive Multi-Million-Token LLM Decoding", fdeinterviews.com, paragraph on KV parallelism):
@@ -21,19 +22,8 @@
 // one group and no consumer can wait on a phase more than one ahead of the one it last consumed.
 // Softmax is online in fp32 and base 2 (scale * log2 e folded into the logits).
 //
-// bf16 KV: TMA tile loads of the page's K and V rows (128-byte swizzle, 8 KiB per 64-column half);
-// ldmatrix feeds the S = q K^T and P V tiles.
-//
-// NVFP4 KV (the pages' simulated results use FP4 KV: paper summary, roofline paragraph). The stage
-// is four 1-D bulk copies of one (page, KV head): K codes, K scales, V codes, V scales (9 KiB at
-// d = 128). E2M1 x E4M3 products are exact in f16 (at most 6 significant bits, 2^-10 .. 2688), so
-// each thread dequantises straight into f16 m16n8k16 fragments: one cvt.rn.f16x2.e2m1x2 and one
-// HMUL2 per two elements. For S = q K^T the MMA's k index is permuted so that a thread's 32
-// contiguous elements of a K row (one 16-byte load) are its B operands for all eight k-steps; q's
-// A fragments use the same permutation. For P V the pool stores V token-pair interleaved (see
-// helix.h), so a byte is already the (token 2i, token 2i+1) pair the B fragment needs, and V's n
-// index is permuted (output column 16 n + j for n-tile j) so one 16-byte load per token pair feeds
-// all sixteen n-tiles; the flush writes O back in natural column order.
+// K and V stream in with TMA tile loads of the page's rows (128-byte swizzle, 8 KiB per 64-column
+// half); ldmatrix feeds the S = q K^T and P V tiles.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -54,18 +44,11 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kChunkBytes = kPage * 64 * 2;  // one 64-column half of a bf16 page-head: 8 KiB
 constexpr int kMergeSlots = 2;               // 16 x D fp32 buffers for the cross-warp merge
 
-enum KvFormat { kBF16 = 0, kNVFP4 = 1 };
-
-template <int D, int FMT>
+template <int D>
 struct GqaCfg {
   static constexpr int NCH = D / 64;  // 64-column halves per bf16 row
-  // NVFP4 stage: K codes | K scales | V codes | V scales of one (page, kv head)
-  static constexpr int KC_BYTES = kPage * D / 2, KS_BYTES = kPage * D / 16;
-  static constexpr int OFF_KS = KC_BYTES, OFF_VC = KC_BYTES + KS_BYTES,
-                       OFF_VS = 2 * KC_BYTES + KS_BYTES;
-  static constexpr int STAGE_BYTES =
-      FMT == kBF16 ? 2 * NCH * kChunkBytes : 2 * (KC_BYTES + KS_BYTES);
-  static constexpr int NSTAGE = FMT == kNVFP4 ? 16 : (D == 128 ? 6 : 10);
+  static constexpr int STAGE_BYTES = 2 * NCH * kChunkBytes;  // K and V of one (page, kv head)
+  static constexpr int NSTAGE = D == 128 ? 6 : 10;
   // floats per workspace segment record: O [16][D], then m, l, lb per row
   static constexpr int REC = kRows * (D + 3);
   static_assert(NSTAGE % kGroups == 0, "a stage must belong to one consumer group");
@@ -83,9 +66,9 @@ struct SmemTail {
   int abort_;
 };
 
-template <int D, int FMT>
+template <int D>
 __host__ __device__ constexpr size_t smem_bytes_for(int units) {
-  return 1024 /*alignment slack*/ + (size_t)GqaCfg<D, FMT>::NSTAGE * GqaCfg<D, FMT>::STAGE_BYTES +
+  return 1024 /*alignment slack*/ + (size_t)GqaCfg<D>::NSTAGE * GqaCfg<D>::STAGE_BYTES +
          (size_t)kMergeSlots * kRows * D * sizeof(float) + sizeof(SmemTail) +
          (size_t)(units + 1) * sizeof(int);
 }
@@ -105,41 +88,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
-// ---- NVFP4 helpers: hardware conversions of packed 4-/8-bit codes to f16x2 (low code -> low half)
-__device__ __forceinline__ void e2m1x4_to_f16x2(uint32_t w, uint32_t& h0, uint32_t& h1,
-                                                uint32_t& h2, uint32_t& h3) {
-  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
-      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
-      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-      : "r"(w));
-}
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
-  return h;
-}
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ float f16_lo_to_f32(uint32_t v) {
-  return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));
-}
-__device__ __forceinline__ float f16_hi_to_f32(uint32_t v) {
-  return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
-}
-
-template <int D, int FMT>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     gqa_partial_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const GqaParams p) {
-  using Cfg = GqaCfg<D, FMT>;
+  using Cfg = GqaCfg<D>;
   constexpr int NCH = Cfg::NCH;
   constexpr int NSTAGE = Cfg::NSTAGE;
   constexpr int KSTEPS = D / 16;  // k-steps of the QK^T contraction
@@ -160,8 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- per-unit page counts and their prefix sums (every CTA computes the same table) ----
   for (int u = tid; u < U; u += kThreads) {
-    const int s = u % p.kvp;
-    const int b = (u / p.kvp) / p.Hkv;
+    const int s = (u + p.u0) % p.kvp;
+    const int b = ((u + p.u0) / p.kvp) / p.Hkv;
     int len = p.shard_lens[s * p.B + b];
     int np = len > 0 ? (len + kPage - 1) / kPage : 0;
     if (np > p.max_pages) {
@@ -205,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Units with no tokens: O_s = 0, lse_s = -inf (handled round-robin by CTA index).
   for (int u = blockIdx.x; u < U; u += gridDim.x) {
     if (pre[u + 1] != pre[u]) continue;
-    const int s = u % p.kvp, bk = u / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
+    const int s = (u + p.u0) % p.kvp, bk = (u + p.u0) / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
     const size_t row0 = ((size_t)s * p.B + b) * p.Hq + (size_t)k * p.G;
     for (int i = tid; i < p.G * D; i += kThreads) p.o_part[row0 * D + i] = 0.f;
     for (int i = tid; i < p.G; i += kThreads) p.lse[row0 + i] = -INFINITY;
@@ -228,11 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ======================================= producer =============================================
   if (warp == kConsumerWarps) {
-    if constexpr (FMT == kBF16) {
-      if (lane == 0) {
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-      }
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
     }
     int u_cur = u_first;  // unit of the first page of the current batch (same in every lane)
     int stage = 0;
@@ -245,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int my_page = -1, my_k = 0, uu = u_cur;
       if (gl < g_end) {
         while (pre[uu + 1] <= gl) ++uu;
-        const int s = uu % p.kvp, bk = uu / p.kvp, b = bk / p.Hkv;
+        const int s = (uu + p.u0) % p.kvp, bk = (uu + p.u0) / p.kvp, b = bk / p.Hkv;
         my_k = bk % p.Hkv;
         my_page = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + (int)(gl - pre[uu]));
       }
@@ -270,23 +221,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               tail->stage_ok[stage] = 1;
               mbar_arrive_expect_tx(&tail->full[stage], Cfg::STAGE_BYTES);
-              if constexpr (FMT == kBF16) {
-                const int row = (page * p.Hkv + k) * kPage;
+              const int row = (page * p.Hkv + k) * kPage;
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) {
-                  tma_load_2d(st + c * kChunkBytes, &tmK, c * 64, row, &tail->full[stage]);
-                  tma_load_2d(st + (NCH + c) * kChunkBytes, &tmV, c * 64, row,
-                              &tail->full[stage]);
-                }
-              } else {
-                const size_t ph = (size_t)page * p.Hkv + k;
-                bulk_load(st, p.k_codes + ph * Cfg::KC_BYTES, Cfg::KC_BYTES, &tail->full[stage]);
-                bulk_load(st + Cfg::OFF_KS, p.k_scale + ph * Cfg::KS_BYTES, Cfg::KS_BYTES,
-                          &tail->full[stage]);
-                bulk_load(st + Cfg::OFF_VC, p.v_codes + ph * Cfg::KC_BYTES, Cfg::KC_BYTES,
-                          &tail->full[stage]);
-                bulk_load(st + Cfg::OFF_VS, p.v_scale + ph * Cfg::KS_BYTES, Cfg::KS_BYTES,
-                          &tail->full[stage]);
+              for (int c = 0; c < NCH; ++c) {
+                tma_load_2d(st + c * kChunkBytes, &tmK, c * 64, row, &tail->full[stage]);
+                tma_load_2d(st + (NCH + c) * kChunkBytes, &tmV, c * 64, row, &tail->full[stage]);
               }
             }
             ++issued;
@@ -324,31 +263,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     lb_run[0] = lb_run[1] = 0.f;
   };
   auto load_q = [&](int u) {
-    const int bk = u / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
+    const int bk = (u + p.u0) / p.kvp, k = bk % p.Hkv, b = bk / p.Hkv;
     const __nv_bfloat16* qb = p.q + ((size_t)b * p.Hq + (size_t)k * p.G) * D;
     const bool v0 = g8 < p.G, v1 = g8 + 8 < p.G;
     const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qb + (size_t)g8 * D);
     const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qb + (size_t)(g8 + 8) * D);
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
-      if constexpr (FMT == kBF16) {
-        const int c0 = 16 * kk + 2 * t4;
-        qa[kk][0] = v0 ? __ldg(r0 + c0 / 2) : 0u;
-        qa[kk][1] = v1 ? __ldg(r1 + c0 / 2) : 0u;
-        qa[kk][2] = v0 ? __ldg(r0 + (c0 + 8) / 2) : 0u;
-        qa[kk][3] = v1 ? __ldg(r1 + (c0 + 8) / 2) : 0u;
-      } else {
-        // permuted k: logical columns (2t, 2t+1 | 2t+8, 2t+9) of k-step kk are head-dim elements
-        // 32t + 4kk + (0, 1 | 2, 3); q is rounded to f16 (exact for |q| >= 2^-14)
-        const int c0 = 32 * t4 + 4 * kk;
-        auto cvt = [](uint32_t bf2) {  // bf16x2 -> f16x2
-          return pack_f16x2(bf16_lo_to_f32(bf2), bf16_hi_to_f32(bf2));
-        };
-        qa[kk][0] = v0 ? cvt(__ldg(r0 + c0 / 2)) : 0u;
-        qa[kk][1] = v1 ? cvt(__ldg(r1 + c0 / 2)) : 0u;
-        qa[kk][2] = v0 ? cvt(__ldg(r0 + c0 / 2 + 1)) : 0u;
-        qa[kk][3] = v1 ? cvt(__ldg(r1 + c0 / 2 + 1)) : 0u;
-      }
+      const int c0 = 16 * kk + 2 * t4;
+      qa[kk][0] = v0 ? __ldg(r0 + c0 / 2) : 0u;
+      qa[kk][1] = v1 ? __ldg(r1 + c0 / 2) : 0u;
+      qa[kk][2] = v0 ? __ldg(r0 + (c0 + 8) / 2) : 0u;
+      qa[kk][3] = v1 ? __ldg(r1 + (c0 + 8) / 2) : 0u;
     }
   };
 
@@ -356,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int u = u_first;
   int s_u = 0, b_u = 0, k_u = 0, len_u = 0;
   auto enter_unit = [&](int uu) {
-    s_u = uu % p.kvp;
-    const int bk = uu / p.kvp;
+    s_u = (uu + p.u0) % p.kvp;
+    const int bk = (uu + p.u0) / p.kvp;
     k_u = bk % p.Hkv;
     b_u = bk / p.Hkv;
     len_u = p.shard_lens[s_u * p.B + b_u];
@@ -389,21 +315,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = stages + (size_t)stage * Cfg::STAGE_BYTES;
         if (tail->stage_ok[stage] && tok0 < nvalid) {
           float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-          if constexpr (FMT == kBF16) {
-            const uint32_t kbase = smem_u32(st);
-            // zero the V rows past the end of the history in this warp's slice (0 * garbage = NaN)
-            if (tok0 + 16 > nvalid) {
-              for (int e = lane; e < 16 * NCH * 8; e += 32) {
-                const int row = tok0 + e / (NCH * 8);
-                const int rem = e % (NCH * 8);
-                if (row >= nvalid)
-                  *reinterpret_cast<uint4*>(st + (NCH + rem / 8) * kChunkBytes + row * 128 +
-                                            (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
-              }
-              fence_proxy_async_smem();
-              __syncwarp();
+          const uint32_t kbase = smem_u32(st);
+          // zero the V rows past the end of the history in this warp's slice (0 * garbage = NaN)
+          if (tok0 + 16 > nvalid) {
+            for (int e = lane; e < 16 * NCH * 8; e += 32) {
+              const int row = tok0 + e / (NCH * 8);
+              const int rem = e % (NCH * 8);
+              if (row >= nvalid)
+                *reinterpret_cast<uint4*>(st + (NCH + rem / 8) * kChunkBytes + row * 128 +
+                                          (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
             }
-            // S = q K^T over this warp's 16 tokens: two n-tiles of 8 tokens
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+          {  // S = q K^T over this warp's 16 tokens: two n-tiles of 8 tokens
             const int token = tok0 + (mi >> 1) * 8 + r8;
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -415,26 +340,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_bf16_16816(s0, qa[kk], b0, b1);
               mma_bf16_16816(s1, qa[kk], b2, b3);
             }
-          } else {
-            // S = q K^T from NVFP4: token g8 of each n-tile, head-dim elements [32 t4, 32 t4 + 32)
-            auto ntile = [&](float(&acc)[4], int token) {
-              const uint4 kc = *reinterpret_cast<const uint4*>(st + token * (D / 2) + t4 * 16);
-              const uint32_t sc2 = e4m3x2_to_f16x2(
-                  *reinterpret_cast<const uint16_t*>(st + Cfg::OFF_KS + token * (D / 16) + 2 * t4));
-              const uint32_t sc_lo = __byte_perm(sc2, 0, 0x1010);  // (s_2t, s_2t)
-              const uint32_t sc_hi = __byte_perm(sc2, 0, 0x3232);  // (s_2t+1, s_2t+1)
-              const uint32_t words[4] = {kc.x, kc.y, kc.z, kc.w};
-#pragma unroll
-              for (int wq = 0; wq < 4; ++wq) {  // word wq holds k-steps 2wq and 2wq+1
-                uint32_t h0, h1, h2, h3;
-                e2m1x4_to_f16x2(words[wq], h0, h1, h2, h3);
-                const uint32_t sc = wq < 2 ? sc_lo : sc_hi;
-                mma_f16_16816(acc, qa[2 * wq], hmul2(h0, sc), hmul2(h1, sc));
-                mma_f16_16816(acc, qa[2 * wq + 1], hmul2(h2, sc), hmul2(h3, sc));
-              }
-            };
-            ntile(s0, tok0 + g8);
-            ntile(s1, tok0 + 8 + g8);
           }
           // online softmax (base 2)
           const int ta = tok0 + 2 * t4, tb = tok0 + 8 + 2 * t4;
@@ -467,25 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run[0] = l_run[0] * al0 + ((pw[0] + pw[1]) + (pw[2] + pw[3]));
           l_run[1] = l_run[1] * al1 + ((pw[4] + pw[5]) + (pw[6] + pw[7]));
           uint32_t pa[4];
-          if constexpr (FMT == kBF16) {
-            pa[0] = pack_bf16x2(pw[0], pw[1]);  // row g,   k 2t..
-            pa[1] = pack_bf16x2(pw[4], pw[5]);  // row g+8, k 2t..
-            pa[2] = pack_bf16x2(pw[2], pw[3]);  // row g,   k 8+2t..
-            pa[3] = pack_bf16x2(pw[6], pw[7]);  // row g+8, k 8+2t..
-            lb_run[0] = lb_run[0] * al0 + (bf16_lo_to_f32(pa[0]) + bf16_hi_to_f32(pa[0])) +
-                        (bf16_lo_to_f32(pa[2]) + bf16_hi_to_f32(pa[2]));
-            lb_run[1] = lb_run[1] * al1 + (bf16_lo_to_f32(pa[1]) + bf16_hi_to_f32(pa[1])) +
-                        (bf16_lo_to_f32(pa[3]) + bf16_hi_to_f32(pa[3]));
-          } else {
-            pa[0] = pack_f16x2(pw[0], pw[1]);
-            pa[1] = pack_f16x2(pw[4], pw[5]);
-            pa[2] = pack_f16x2(pw[2], pw[3]);
-            pa[3] = pack_f16x2(pw[6], pw[7]);
-            lb_run[0] = lb_run[0] * al0 + (f16_lo_to_f32(pa[0]) + f16_hi_to_f32(pa[0])) +
-                        (f16_lo_to_f32(pa[2]) + f16_hi_to_f32(pa[2]));
-            lb_run[1] = lb_run[1] * al1 + (f16_lo_to_f32(pa[1]) + f16_hi_to_f32(pa[1])) +
-                        (f16_lo_to_f32(pa[3]) + f16_hi_to_f32(pa[3]));
-          }
+          pa[0] = pack_bf16x2(pw[0], pw[1]);  // row g,   k 2t..
+          pa[1] = pack_bf16x2(pw[4], pw[5]);  // row g+8, k 2t..
+          pa[2] = pack_bf16x2(pw[2], pw[3]);  // row g,   k 8+2t..
+          pa[3] = pack_bf16x2(pw[6], pw[7]);  // row g+8, k 8+2t..
+          lb_run[0] = lb_run[0] * al0 + (bf16_lo_to_f32(pa[0]) + bf16_hi_to_f32(pa[0])) +
+                      (bf16_lo_to_f32(pa[2]) + bf16_hi_to_f32(pa[2]));
+          lb_run[1] = lb_run[1] * al1 + (bf16_lo_to_f32(pa[1]) + bf16_hi_to_f32(pa[1])) +
+                      (bf16_lo_to_f32(pa[3]) + bf16_hi_to_f32(pa[3]));
           if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
@@ -495,50 +389,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               O[j][3] *= al1;
             }
           }
-          if constexpr (FMT == kBF16) {
-            // O += P V over the 16 tokens: V^T fragments via transposing ldmatrix
-            const uint32_t vbase = smem_u32(st) + NCH * kChunkBytes;
-            const int token = tok0 + (mi & 1) * 8 + r8;
+          // O += P V over the 16 tokens: V^T fragments via transposing ldmatrix
+          const uint32_t vbase = smem_u32(st) + NCH * kChunkBytes;
+          const int token = tok0 + (mi & 1) * 8 + r8;
 #pragma unroll
-            for (int n2 = 0; n2 < NT / 2; ++n2) {
-              const int dch = 2 * n2 + (mi >> 1);
-              const uint32_t addr = vbase + (dch >> 3) * kChunkBytes + token * 128 +
-                                    ((((dch & 7) ^ (token & 7))) << 4);
-              uint32_t v0, v1, v2, v3;
-              ldsm_x4_trans(addr, v0, v1, v2, v3);
-              mma_bf16_16816(O[2 * n2], pa, v0, v1);
-              mma_bf16_16816(O[2 * n2 + 1], pa, v2, v3);
-            }
-          } else {
-            // O += P V from NVFP4: token pairs (2t, 2t+1) and (2t+8, 2t+9) of the slice, output
-            // columns 16 g8 + j (n-tile j). A pair row's 16-byte chunks are stored XOR-swizzled by
-            // 2 (pair mod 4), which spreads the eight lanes of a quarter-warp over all banks. The
-            // scales of tokens past the history are zeroed so their codes contribute nothing.
-            const uint8_t* vc = st + Cfg::OFF_VC;
-            const uint8_t* vsc = st + Cfg::OFF_VS + g8 * kPage;
-            const int pa_ = tok0 / 2 + t4, pb_ = tok0 / 2 + t4 + 4;
-            const uint4 va = *reinterpret_cast<const uint4*>(vc + pa_ * D +
-                                                             ((g8 ^ ((pa_ & 3) << 1)) << 4));
-            const uint4 vb = *reinterpret_cast<const uint4*>(vc + pb_ * D +
-                                                             ((g8 ^ ((pb_ & 3) << 1)) << 4));
-            uint32_t sa = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc + ta));
-            uint32_t sb = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc + tb));
-            const uint32_t ma = (ta < nvalid ? 0x0000ffffu : 0u) | (ta + 1 < nvalid ? 0xffff0000u : 0u);
-            const uint32_t mb = (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
-            sa &= ma;
-            sb &= mb;
-            const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-            const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-            for (int wq = 0; wq < 4; ++wq) {
-              uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-              e2m1x4_to_f16x2(wa[wq], a0, a1, a2, a3);
-              e2m1x4_to_f16x2(wb[wq], c0, c1, c2, c3);
-              mma_f16_16816(O[4 * wq + 0], pa, hmul2(a0, sa), hmul2(c0, sb));
-              mma_f16_16816(O[4 * wq + 1], pa, hmul2(a1, sa), hmul2(c1, sb));
-              mma_f16_16816(O[4 * wq + 2], pa, hmul2(a2, sa), hmul2(c2, sb));
-              mma_f16_16816(O[4 * wq + 3], pa, hmul2(a3, sa), hmul2(c3, sb));
-            }
+          for (int n2 = 0; n2 < NT / 2; ++n2) {
+            const int dch = 2 * n2 + (mi >> 1);
+            const uint32_t addr = vbase + (dch >> 3) * kChunkBytes + token * 128 +
+                                  ((((dch & 7) ^ (token & 7))) << 4);
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_trans(addr, v0, v1, v2, v3);
+            mma_bf16_16816(O[2 * n2], pa, v0, v1);
+            mma_bf16_16816(O[2 * n2 + 1], pa, v2, v3);
           }
         }
         __syncwarp();
@@ -623,10 +485,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           add(1);
 #pragma unroll
           for (int j = 0; j < NT; ++j) {  // natural [row][column] layout into slot 0
-            // n-tile j, fragment columns 2t, 2t+1 are head-dim columns 8j + 2t (+1) for bf16 and
-            // 16 (2t) + j, 16 (2t + 1) + j for NVFP4 (its permuted n index)
-            const int ca = FMT == kBF16 ? 8 * j + 2 * t4 : 32 * t4 + j;
-            const int cb = FMT == kBF16 ? ca + 1 : 32 * t4 + 16 + j;
+            // n-tile j, fragment columns 2t, 2t+1 are head-dim columns 8j + 2t (+1)
+            const int ca = 8 * j + 2 * t4;
+            const int cb = ca + 1;
             float* r0 = Obuf + g8 * D;
             r0[ca] = O[j][0];
             r0[cb] = O[j][1];
@@ -737,11 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D, int FMT>
+template <int D>
 static helix_status launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const GqaParams& p,
                            int grid, cudaStream_t stream) {
-  const size_t smem = smem_bytes_for<D, FMT>(p.units);
-  auto kern = gqa_partial_kernel<D, FMT>;
+  const size_t smem = smem_bytes_for<D>(p.units);
+  auto kern = gqa_partial_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return HELIX_ERR_CUDA;
@@ -749,26 +610,19 @@ static helix_status launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const
   return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
 }
 
-size_t gqa_partial_smem_bytes(int head_dim, int nvfp4, int units) {
-  if (nvfp4) return smem_bytes_for<128, kNVFP4>(units);
-  return head_dim == 64 ? smem_bytes_for<64, kBF16>(units) : smem_bytes_for<128, kBF16>(units);
+size_t gqa_partial_smem_bytes(int head_dim, int units) {
+  return head_dim == 64 ? smem_bytes_for<64>(units) : smem_bytes_for<128>(units);
 }
 
 size_t gqa_segment_record_floats(int head_dim) {
-  return head_dim == 64 ? GqaCfg<64, kBF16>::REC : GqaCfg<128, kBF16>::REC;
+  return head_dim == 64 ? GqaCfg<64>::REC : GqaCfg<128>::REC;
 }
 
 helix_status gqa_partial_bf16_launch(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                      const GqaParams& p, int grid, cudaStream_t stream) {
-  if (p.D == 128) return launch<128, kBF16>(tmK, tmV, p, grid, stream);
-  if (p.D == 64) return launch<64, kBF16>(tmK, tmV, p, grid, stream);
+  if (p.D == 128) return launch<128>(tmK, tmV, p, grid, stream);
+  if (p.D == 64) return launch<64>(tmK, tmV, p, grid, stream);
   return HELIX_ERR_UNSUPPORTED;
-}
-
-helix_status gqa_partial_nvfp4_launch(const GqaParams& p, int grid, cudaStream_t stream) {
-  if (p.D != 128) return HELIX_ERR_UNSUPPORTED;
-  CUtensorMap unused{};
-  return launch<128, kNVFP4>(unused, unused, p, grid, stream);
 }
 
 }  // namespace helix

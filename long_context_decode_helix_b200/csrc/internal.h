@@ -26,11 +26,14 @@ struct GqaParams {
   const uint8_t* k_codes;     // NVFP4 only: [pages][Hkv][64][D/2]
   const uint8_t* v_codes;
   int B, Hq, Hkv, G, D, kvp, max_pages, num_pages, units;
+  int u0;                     // first unit of this launch (a request boundary)
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-size_t gqa_partial_smem_bytes(int head_dim, int nvfp4, int units);
+size_t gqa_partial_smem_bytes(int head_dim, int units);  // bf16 kernel
 size_t gqa_segment_record_floats(int head_dim);
+size_t gqa_nvfp4_smem_bytes(int units);                  // NVFP4 kernel (head_dim 128)
+size_t gqa_nvfp4_segment_record_floats();
 helix_status gqa_partial_bf16_launch(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                      const GqaParams& p, int grid, cudaStream_t stream);
 helix_status gqa_partial_nvfp4_launch(const GqaParams& p, int grid, cudaStream_t stream);
@@ -45,6 +48,7 @@ struct MlaParams {
   float* seg;                 // [clusters][2 slots][2 halves][record]
   uint32_t* err;              // may be null
   int B, kvp, max_pages, num_pages, units;
+  int u0;                     // first unit of this launch (a request boundary)
   float scale_log2;
 };
 size_t mla_partial_smem_bytes(int units);
@@ -67,8 +71,9 @@ struct AppendParams {
 };
 helix_status append_launch(const AppendParams& p, cudaStream_t stream);
 
-helix_status combine_launch(int kvp, int batch, int num_q_heads, int v_dim, const float* o_partial,
-                            const float* lse, void* o_out, int o_dtype, float* lse_out,
-                            cudaStream_t stream);
+// rows = B * Hq (the shard stride of o_partial / lse); combines rows [row0, row0 + nrows)
+helix_status combine_launch(int kvp, int rows, int row0, int nrows, int v_dim,
+                            const float* o_partial, const float* lse, void* o_out, int o_dtype,
+                            float* lse_out, cudaStream_t stream);
 
 }  // namespace helix

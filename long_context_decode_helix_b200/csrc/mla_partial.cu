@@ -15,16 +15,24 @@
 //   * CTA r keeps half of q's contraction (head-dim elements [288 r, 288 r + 288)) in shared memory
 //     and computes a partial score tile S_r = q[:, half] C[:, half]^T (M = 128 heads, N = 32 tokens,
 //     K = 288) into TMEM;
-//   * the two CTAs swap their partials through distributed shared memory (plain remote stores and
-//     remote mbarrier arrivals -- no multicast loads), so both hold the same full S;
-//   * each CTA runs the same online softmax and accumulates O for its half of the value columns
-//     (M = 128, N = 256, K = 32 tokens) in 256 TMEM columns, reading V straight from the latent tile
-//     it already holds (MN-major operand).
+//   * the two CTAs swap their partials through distributed shared memory: st.async stores into the
+//     peer's exchange buffer complete a transaction count on the peer's mbarrier, and the buffer is
+//     handed back with a relaxed remote arrive (no multicast loads anywhere), so both hold the same
+//     full S;
+//   * each CTA runs the same online softmax, writes P (bf16) back into TMEM and accumulates O for
+//     its half of the value columns (M = 128, N = 256, K = 32 tokens) in 256 TMEM columns with the
+//     TS form of the MMA (A = P from TMEM, B = V read straight from the latent tile it already holds,
+//     MN-major).
 // Each CTA loads five 64-column chunks of every latent row (chunks 0-4 or 4-8), so together the pair
 // reads the 576-wide row once plus one 64-column chunk.
 //
-// Warps: 0-3 softmax / epilogue (thread i owns head i = TMEM lane i), 4 TMA producer, 5 MMA issuer
-// (one elected thread) and TMEM allocator. O is rescaled lazily: the exponent base only moves when
+// Warps: 0-7 softmax / epilogue in two groups of four (group g takes the tiles i with i % 2 == g,
+// so two tiles are in the softmax at once; thread h of a group owns head h = TMEM lane h), 8 TMA
+// producer, 9 MMA issuer (one elected thread, which issues whichever of the next S tile or the next
+// P V product is ready) and TMEM allocator. Score tiles have four TMEM buffers, so the tensor core
+// runs ahead of the softmax. The groups share one reference maximum per head, handed from the owner
+// of tile i-1 to the owner of tile i through shared memory and a named barrier; each group keeps its
+// own running sum, and the two are merged at the end of a segment. O is rescaled lazily: the exponent base only moves when
 // a row maximum grows by more than 8 (in base-2 units), so weights stay below 2^8 and the 256-column
 // TMEM rescale is rare. Work is split over the (request, shard) units exactly as in the GQA kernel:
 // each cluster takes an equal contiguous range of 32-token tiles; split units are merged by the last
@@ -42,7 +50,7 @@ namespace helix {
 namespace {
 
 constexpr int kHeads = 128;
-constexpr int kDK = 576, kDV = 512, kHalfDV = 256;
+constexpr int kDV = 512, kHalfDV = 256;  // V: the first 512 of the 576 latent columns
 constexpr int kTok = 32;                   // tokens per tile
 constexpr int kPageTok = 64;               // tokens per page
 constexpr int kChunks = 5;                 // 64-column chunks of a latent row per CTA
@@ -51,20 +59,29 @@ constexpr int kNS = 5;                     // tile stages
 constexpr int kNX = 2;                     // score-exchange buffers
 constexpr int kStageBytes = kTok * kChunks * 128;     // 20 KiB
 constexpr int kQBytes = kHeads * kChunks * 128;        // 80 KiB
-constexpr uint32_t kSCol = 256, kPCol = 320;           // TMEM columns: O [0,256), S 2x32, P 2x16
+constexpr int kSBuf = 4;                               // score-tile buffers in TMEM
+constexpr uint32_t kSCol = 256, kPCol = 384;           // TMEM columns: O [0,256), S 4x32, P 2x16
 constexpr int kXStride = kTok + 4;                     // padded fp32 row of the exchange buffer
 constexpr int kXBytes = kHeads * kXStride * 4;         // 18 KiB
-constexpr int kThreads = 6 * 32;
+// warps 0-7: two softmax groups of four (group g takes the tiles i with i % 2 == g)
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 10 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRec = kHeads * (kHalfDV + 3);           // floats per segment record (one half)
 
 struct MlaTail {
   uint64_t stage_full[kNS], stage_empty[kNS];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[kSBuf], s_empty[kSBuf];
   uint64_t p_full[2], p_empty[2];
   uint64_t x_full[kNX], x_free[kNX];
   uint64_t q_full, q_empty;
   int stage_ok[kNS];
+  uint64_t m_ready[2][4];   // [publishing group][32-row slice]: mpub holds its latest maximum
+  uint64_t seg_ready;       // segment end: the non-owning group has stored its (m, l)
+  uint64_t o_drained;       // segment end: the owning group has read O out of TMEM
+  float mpub[kHeads];       // reference maximum after the latest tile, handed between groups
+  float seg_m[2][kHeads];   // per group: the maximum its running sum is relative to
+  float seg_l[2][kHeads];   // per group: running sum of the weights of its tiles
   uint32_t tmem_base;
   int flag;
   int abort_;
@@ -213,7 +230,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 
 // Shared-memory matrix descriptor (sm_100 format): start, leading and stride byte offsets in
 // 16-byte units, descriptor version 1, swizzle mode in the top three bits.
-constexpr uint64_t kSwizzle128 = 2, kSwizzle64 = 4;
+constexpr uint64_t kSwizzle128 = 2;
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
                                               uint32_t sbo_bytes, uint64_t swizzle) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
@@ -254,7 +271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // ---- tiles per unit and their prefix sums ----
   for (int u = tid; u < U; u += kThreads) {
-    const int s = u % p.kvp, b = u / p.kvp;
+    const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
     int len = p.shard_lens[s * p.B + b];
     if (len > p.max_pages * kPageTok) {
       if (blockIdx.x == 0) raise_dev_error(p.err, HELIX_DEVERR_CAPACITY);
@@ -268,16 +285,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&tail->stage_full[i], 1);
       mbar_init(&tail->stage_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&tail->s_full[i], 1);
-      mbar_init(&tail->s_empty[i], 4);  // one arrival per softmax warp
+      mbar_init(&tail->s_empty[i], 4);  // one arrival per warp of the group that reads it
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&tail->p_full[i], 4);
       mbar_init(&tail->p_empty[i], 1);
+      for (int j = 0; j < 4; ++j) mbar_init(&tail->m_ready[i][j], 32);  // every lane of a warp
     }
+    mbar_init(&tail->seg_ready, kHeads);  // every thread of a group
+    mbar_init(&tail->o_drained, kHeads);
     for (int i = 0; i < kNX; ++i) {
       // x_full: armed by this CTA with the expected bytes, completed by the peer's async stores
       mbar_init(&tail->x_full[i], 1);
-      mbar_init(&tail->x_free[i], 4);  // one arrival per softmax warp of the peer CTA
+      mbar_init(&tail->x_free[i], 4);  // one arrival per warp of the peer CTA's group
     }
     mbar_init(&tail->q_full, 1);
     mbar_init(&tail->q_empty, 1);
@@ -287,7 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // arm the exchange barriers for the first kNX tiles (128 rows x 32 fp32 scores each)
     for (int i = 0; i < kNX; ++i) mbar_arrive_expect_tx(&tail->x_full[i], kHeads * kTok * 4);
   }
-  if (warp == 5) {  // allocate all 512 TMEM columns (one CTA per SM)
+  if (warp == kMmaWarp) {  // allocate all 512 TMEM columns (one CTA per SM)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&tail->tmem_base)),
                  "r"(kTmemCols)
@@ -322,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // units with no tokens: O_s = 0, lse_s = -inf (this CTA's value half)
   for (int u = pair; u < U; u += npairs) {
     if (pre[u + 1] != pre[u]) continue;
-    const int s = u % p.kvp, b = u / p.kvp;
+    const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
     const size_t row0 = ((size_t)s * p.B + b) * kHeads;
     for (int i = tid; i < kHeads * kHalfDV; i += kThreads)
       p.o_part[(row0 + i / kHalfDV) * kDV + rank * kHalfDV + i % kHalfDV] = 0.f;
@@ -344,7 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (pre[u_first + 1] <= g_begin) ++u_first;
   }
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ===================================== TMA producer ========================================
     if (lane == 0 && active) {
       prefetch_tensormap(&tmC);
@@ -355,7 +377,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (long long g = g_begin; g < g_end; ++g) {
         if (*(volatile int*)&tail->abort_) break;
         while (pre[u + 1] <= g) ++u;
-        const int s = u % p.kvp, b = u / p.kvp;
+        const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
         if (u != cur) {  // (re)load this CTA's half of q for request b
           if (qcount > 0 && !mbar_wait(&tail->q_empty, (qcount - 1) & 1)) {
             raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
@@ -392,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (++stage == kNS) { stage = 0; ++round; }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ====================================== MMA issuer =========================================
     if (lane == 0 && active) {
       // Event-driven issue: the next score tile S(ns) goes out as soon as its stage has landed and
@@ -440,9 +462,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             cur = u_s;
             ++qcount;
           }
-          const int st = (int)(ns % kNS), sb = (int)(ns & 1);
+          const int st = (int)(ns % kNS), sb = (int)(ns % kSBuf);
           if (u_s == cur && mbar_test(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) &&
-              (ns < 2 || mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - 2) >> 1) & 1)))) {
+              (ns < kSBuf ||
+               mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - kSBuf) / kSBuf) & 1)))) {
             tc_fence_after();
             // S_partial = q[:, half] C_tile[:, half]^T: 18 k-steps of 16 over this CTA's columns
             // Descriptors are built once per tile; a k-step only advances the start address
@@ -486,35 +509,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ================================= softmax / epilogue warps ================================
-    const int h = tid;  // head row = TMEM lane
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    // Two groups of four warps; group grp takes the tiles i with i % 2 == grp, so two tiles are
+    // in the softmax at once. Thread h of either group owns head row h (TMEM lane h). The groups
+    // share one reference maximum per row: the owner of tile i decides it from the value the
+    // other group left after tile i-1 and hands it on through mpub and an mbarrier per 32-row
+    // slice; each group keeps its own running sum, relative to the maximum it last saw, and the
+    // two sums are merged when a segment ends. Every wait between the groups is a bounded
+    // mbarrier wait: each barrier completes one phase per hand-over, and neither side can get a
+    // phase ahead (the next hand-over in one direction needs the one in the other).
+    const int grp = warp >> 2, slice = warp & 3;
+    const int h = tid & (kHeads - 1);
+    const uint32_t tl = tmem + ((uint32_t)(slice * 32) << 16);
+    int n_seg = 0;  // segment ends this group has gone through
     const float sl2 = p.scale_log2;
-    float m_use = -INFINITY, l_run = 0.f, lb_run = 0.f;
-    bool has_o = false;  // O holds a partial sum for the current segment
+    float m_own = -INFINITY, l_own = 0.f;  // this group's running sum and its reference maximum
     bool dead = !active;
-    int u = u_first;
-    long long seg_begin = g_begin;
     const uint32_t x_peer = map_peer(smem_u32(x_s), peer);
     const uint32_t xfull_peer = map_peer(smem_u32(&tail->x_full[0]), peer);
     const uint32_t xfree_peer = map_peer(smem_u32(&tail->x_free[0]), peer);
+    const long long n_tiles = g_end - g_begin;
     // warp-uniform bounded waits: tcgen05.ld / st below are warp-collective
     auto wwait = [&](uint64_t* bar, uint32_t parity, bool cluster_scope) {
       if (dead) return;
       const bool ok = cluster_scope ? mbar_wait_cluster(bar, parity) : mbar_wait(bar, parity);
       if (!__all_sync(0xffffffffu, ok)) dead = true;
     };
-    // Phase A(j): read tile j's partial scores from TMEM and send them to the peer.
-    // Phase B(i): receive the peer's partial for tile i, finish the softmax, hand P to the MMA.
-    // The loop runs A(i+1) before B(i), so the exchange of tile i overlaps the work on tile i+1.
-    auto phase_a = [&](long long j, float (&sv)[32], bool& tile_ok) {
-      const int sb = (int)(j & 1), xb = (int)(j % kNX);
-      const int st_j = (int)(j % kNS);
+    int u = u_first;            // unit of the tile in hand
+    int len_u = 0, cur_u = -1;  // its history length (read once per unit)
+    auto unit_of = [&](long long g) {
+      while (pre[u + 1] <= g) ++u;
+      if (u != cur_u) {
+        cur_u = u;
+        len_u = p.shard_lens[((u + p.u0) % p.kvp) * p.B + (u + p.u0) / p.kvp];
+      }
+    };
+    // Segment end at a tile of the other group: hand it this group's running (m, l) (seg_ready),
+    // then wait until it has read O out of TMEM (o_drained), since this group's next P V would
+    // overwrite O.
+    auto join_segment_end = [&]() {
+      tail->seg_m[grp][h] = m_own;
+      tail->seg_l[grp][h] = l_own;
+      mbar_arrive(&tail->seg_ready);
+      wwait(&tail->o_drained, (uint32_t)(n_seg & 1), false);
+      ++n_seg;
+      m_own = -INFINITY;
+      l_own = 0.f;
+    };
+    float sv[32];
+    for (long long i = grp; i < n_tiles; i += 2) {
+      const long long g = g_begin + i;
+      unit_of(g);
+      const bool fresh = g == g_begin || g == pre[u];  // first tile of a segment
+      const bool seg_end = g + 1 == g_end || g + 1 == pre[u + 1];
+      const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
+      const int lt = (int)(g - pre[u]);
+      const int nvalid = min(kTok, len_u - lt * kTok);
+      const int sb = (int)(i % kSBuf), st_i = (int)(i % kNS);
+      // ---- A: this CTA's partial scores of tile i, from TMEM to the peer's exchange buffer ----
       dead = __any_sync(0xffffffffu, dead || *(volatile int*)&tail->abort_ != 0);
-      wwait(&tail->s_full[sb], (uint32_t)((j >> 1) & 1), false);
+      wwait(&tail->s_full[sb], (uint32_t)((i / kSBuf) & 1), false);
       // also observe the tile's load barrier: orders the stage's validity flag and its data before
-      // the zeroing of rows past the end of the history in phase B
-      wwait(&tail->stage_full[st_j], (uint32_t)((j / kNS) & 1), false);
-      tile_ok = tail->stage_ok[st_j] != 0;
+      // the zeroing of rows past the end of the history below
+      wwait(&tail->stage_full[st_i], (uint32_t)((i / kNS) & 1), false);
+      const bool tile_ok = tail->stage_ok[st_i] != 0;
       if (!dead) {
         tc_fence_after();
         tmem_ld32(tl + kSCol + sb * kTok, sv);
@@ -525,24 +582,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->s_empty[sb]);
-      if (j >= kNX) wwait(&tail->x_free[xb], (uint32_t)(((j - kNX) / kNX) & 1), true);
-      const uint32_t dst = x_peer + (uint32_t)((xb * kHeads + h) * kXStride * 4);
-#pragma unroll
-      for (int c = 0; c < kTok; c += 4)
-        st_async_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3], xfull_peer + xb * 8);
-    };
-    long long i = 0;
-    auto phase_b = [&](float (&sv)[32], bool tile_ok) -> bool {  // returns true at a segment end
-      const long long g = g_begin + i;
-      while (pre[u + 1] <= g) ++u;
-      const int s = u % p.kvp, b = u / p.kvp;
-      const int lt = (int)(g - pre[u]);
-      const int len = p.shard_lens[s * p.B + b];
-      const int nvalid = min(kTok, len - lt * kTok);
-      const int xb = (int)(i % kNX), pb = (int)(i & 1);
-      wwait(&tail->x_full[xb], (uint32_t)((i / kNX) & 1), true);
+      if (i >= 2) wwait(&tail->x_free[grp], (uint32_t)(((i - 2) >> 1) & 1), true);
       {
-        const float* mine = x_s + (size_t)(xb * kHeads + h) * kXStride;
+        const uint32_t dst = x_peer + (uint32_t)((grp * kHeads + h) * kXStride * 4);
+#pragma unroll
+        for (int c = 0; c < kTok; c += 4)
+          st_async_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3], xfull_peer + grp * 8);
+      }
+      // the previous tile closed a segment owned by the other group: join its flush before this
+      // tile's P can reach the MMA (its P V would overwrite O)
+      if (fresh && i > 0) join_segment_end();
+      // ---- B: add the peer's partial, softmax, P into TMEM ----
+      wwait(&tail->x_full[grp], (uint32_t)((i >> 1) & 1), true);
+      {
+        const float* mine = x_s + (size_t)(grp * kHeads + h) * kXStride;
 #pragma unroll
         for (int c = 0; c < kTok; c += 4) {
           const float4 v = *reinterpret_cast<const float4*>(mine + c);
@@ -552,14 +605,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           sv[c + 3] += v.w;
         }
       }
-      // re-arm this buffer's barrier for tile i+2 (once every thread here has observed tile i's
-      // phase, which the wait above guarantees for this thread), then release the buffer
-      if (h == 0 && i + kNX < g_end - g_begin)
-        mbar_arrive_expect_tx(&tail->x_full[xb], kHeads * kTok * 4);
-      keep_alive(sv);  // the buffer's loads have returned before the buffer is handed back
+      // re-arm this group's exchange barrier for tile i+2 (every thread here has observed tile
+      // i's phase), then hand the buffer back to the peer once its loads have returned
+      if (h == 0 && i + 2 < n_tiles) mbar_arrive_expect_tx(&tail->x_full[grp], kHeads * kTok * 4);
+      keep_alive(sv);
       __syncwarp();
-      if (lane == 0) remote_arrive_relaxed(xfree_peer + xb * 8);
-      // ---- online softmax (base 2), lazy rescale ----
+      if (lane == 0) remote_arrive_relaxed(xfree_peer + grp * 8);
       if (nvalid == kTok && tile_ok) {
 #pragma unroll
         for (int c = 0; c < kTok; ++c) sv[c] *= sl2;
@@ -580,24 +631,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       // V rows past the end of the history are zeroed before the P V product reads them
       if (nvalid < kTok && !dead) {
-        uint8_t* st = stage_s + (i % kNS) * kStageBytes;
+        uint8_t* stg = stage_s + st_i * kStageBytes;
         for (int e = h; e < (kTok - nvalid) * 4 * 8; e += kHeads) {
           const int row = nvalid + e / 32, rem = e % 32;
-          *reinterpret_cast<uint4*>(st + (rem / 8) * kTok * 128 + row * 128 + (rem % 8) * 16) =
+          *reinterpret_cast<uint4*>(stg + (rem / 8) * kTok * 128 + row * 128 + (rem % 8) * 16) =
               make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
-      bool rescale = false;
-      float alpha = 1.f;
-      if (!has_o) {
-        if (mx > -INFINITY) m_use = mx;
-      } else if (mx > m_use + 8.f) {
-        alpha = fast_exp2(m_use - mx);
-        m_use = mx;
-        rescale = true;
+      // ---- the shared reference maximum: from the other group's tile i-1, lazily raised ----
+      float m_prev = -INFINITY;
+      if (i > 0) {  // the other group published after tile i-1 (its ((i-1) >> 1)-th hand-over)
+        wwait(&tail->m_ready[grp ^ 1][slice], (uint32_t)(((i - 1) >> 1) & 1), false);
+        if (!fresh) m_prev = tail->mpub[h];
       }
-      const float mb = m_use == -INFINITY ? 0.f : m_use;
+      float m_new = m_prev;
+      if (m_prev == -INFINITY) m_new = mx;
+      else if (mx > m_prev + 8.f) m_new = mx;
+      const bool rescale = m_prev != -INFINITY && m_new > m_prev;  // O holds tiles so far
+      if (i + 1 < n_tiles) {
+        tail->mpub[h] = m_new;
+        mbar_arrive(&tail->m_ready[grp][slice]);
+      }
+      const float mb = m_new == -INFINITY ? 0.f : m_new;
+      if (m_own != m_new) {  // this group's sum moves to the new reference
+        l_own = l_own > 0.f ? l_own * fast_exp2(m_own - mb) : 0.f;
+        m_own = m_new;
+      }
       uint32_t pk[16];
       float ps[16];
 #pragma unroll
@@ -611,12 +671,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
       // O is normalised by the fp32 sum (the bf16-rounded weights differ from it by < 2^-9)
-      const float psum = (ps[0] + ps[2]) + (ps[1] + ps[3]);
-      const float pbsum = psum;
-      // P(i) goes into buffer pb, last read by PV(i-2); a rescale also needs PV(i-1) finished
-      if (i >= 2) wwait(&tail->p_empty[pb], (uint32_t)(((i - 2) >> 1) & 1), false);
+      l_own += (ps[0] + ps[2]) + (ps[1] + ps[3]);
+      // P(i) goes into this group's buffer, last read by PV(i-2)
+      if (i >= 2) wwait(&tail->p_empty[grp], (uint32_t)(((i - 2) >> 1) & 1), false);
       if (__any_sync(0xffffffffu, rescale) && !dead) {
-        if (i >= 1) wwait(&tail->p_empty[pb ^ 1], (uint32_t)(((i - 1) >> 1) & 1), false);
+        // O holds tiles < i: wait for PV(i-1) (the other group's), then rescale the rows that
+        // moved. PV(i+1) cannot start before P(i) is handed over, which comes after this.
+        if (i >= 1) wwait(&tail->p_empty[grp ^ 1], (uint32_t)(((i - 1) >> 1) & 1), false);
+        const float alpha = rescale ? fast_exp2(m_prev - m_new) : 1.f;
         tc_fence_after();
         for (int c = 0; c < kHalfDV; c += 32) {
           float o[32];
@@ -627,52 +689,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
       }
-      if (rescale) {
-        l_run *= alpha;
-        lb_run *= alpha;
-      }
-      l_run += psum;
-      lb_run += pbsum;
-      has_o = true;
       // P row h (32 bf16) into this thread's TMEM lane: the A operand of the P V product
-      if (!dead) tmem_st16(tl + kPCol + pb * 16, pk);
+      if (!dead) tmem_st16(tl + kPCol + grp * 16, pk);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tail->p_full[pb]);
-      return g + 1 == g_end || g + 1 == pre[u + 1];
-    };
-    const long long n_tiles = g_end - g_begin;
-    float sv0[32], sv1[32];
-    bool ok0 = false, ok1 = false;
-    if (n_tiles > 0) phase_a(0, sv0, ok0);
-    for (i = 0; i < n_tiles; ++i) {
-      bool seg_end;
-      if ((i & 1) == 0) {
-        if (i + 1 < n_tiles) phase_a(i + 1, sv1, ok1);
-        seg_end = phase_b(sv0, ok0);
-      } else {
-        if (i + 1 < n_tiles) phase_a(i + 1, sv0, ok0);
-        seg_end = phase_b(sv1, ok1);
-      }
-      const long long g = g_begin + i;
-      const int s = u % p.kvp, b = u / p.kvp;
-      const int pb = (int)(i & 1);
-      const uint32_t ph = (uint32_t)((i >> 1) & 1);
+      if (lane == 0) mbar_arrive(&tail->p_full[grp]);
 
-      // ---- end of a segment ----
-      if (seg_end) {
+      if (!seg_end) continue;
+      // ---- end of a segment (this group owns its last tile) ----
+      wwait(&tail->seg_ready, (uint32_t)(n_seg & 1), false);  // the other group's (m, l)
+      {
         // O is complete once PV(i) has finished
-        wwait(&tail->p_empty[pb], ph, false);
+        wwait(&tail->p_empty[grp], (uint32_t)((i >> 1) & 1), false);
         tc_fence_after();
+        const float M = m_own;  // the reference of this tile: the segment's final maximum
+        const float Mb = M == -INFINITY ? 0.f : M;
+        const int o_grp = grp ^ 1;
+        const float m_o = tail->seg_m[o_grp][h], l_o = tail->seg_l[o_grp][h];
+        const float l_run = l_own + (l_o > 0.f ? l_o * fast_exp2(m_o - Mb) : 0.f);
         const size_t orow = ((size_t)s * p.B + b) * kHeads + h;
-        const bool whole = seg_begin == pre[u] && g + 1 == pre[u + 1];
-        const float M = m_use;
+        const bool whole = g_begin <= pre[u] && g + 1 == pre[u + 1];
         float* rec = nullptr;
         if (!whole) {
           const int slot = (g_begin >= pre[u]) ? 0 : 1;
           rec = p.seg + (((size_t)pair * 2 + slot) * 2 + rank) * kRec;
         }
-        const float inv = lb_run > 0.f ? 1.f / lb_run : 0.f;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         for (int c = 0; c < kHalfDV; c += 32) {
           float o[32];
           if (!dead) tmem_ld32(tl + c, o);
@@ -692,15 +734,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         } else {
           rec[kHeads * kHalfDV + h] = M;
           rec[kHeads * kHalfDV + kHeads + h] = l_run;
-          rec[kHeads * kHalfDV + 2 * kHeads + h] = lb_run;
+          rec[kHeads * kHalfDV + 2 * kHeads + h] = l_run;
           __threadfence();
-          named_barrier_sync(1, kHeads);
+          named_barrier_sync(2 + grp, kHeads);
           const int c_lo = cta_of(pre[u], W, Geff), c_hi = cta_of((long long)pre[u + 1] - 1, W, Geff);
           if (h == 0) {
             const int ticket = atomicAdd(&p.tickets[u * 2 + rank], 1);
             tail->flag = ticket == c_hi - c_lo;
           }
-          named_barrier_sync(1, kHeads);
+          named_barrier_sync(2 + grp, kHeads);
           if (tail->flag) {  // merge every cluster's segment of this unit, for this value half
             __threadfence();
             float Mm = -INFINITY;
@@ -735,24 +777,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                   make_float4(acc.x * invm, acc.y * invm, acc.z * invm, acc.w * invm);
             }
             if (rank == 0) p.lse[orow] = Lm > 0.f ? (Mm + log2f(Lm)) * kLn2 : -INFINITY;
-            named_barrier_sync(1, kHeads);
+            named_barrier_sync(2 + grp, kHeads);
             if (h == 0) p.tickets[u * 2 + rank] = 0;
           }
         }
-        named_barrier_sync(1, kHeads);
-        m_use = -INFINITY;
-        l_run = lb_run = 0.f;
-        has_o = false;
-        seg_begin = g + 1;
       }
+      mbar_arrive(&tail->o_drained);
+      ++n_seg;
+      m_own = -INFINITY;
+      l_own = 0.f;
     }
+    // the range's last tile belongs to the other group: join its flush
+    if (n_tiles > 0 && ((n_tiles - 1) & 1) != grp) join_segment_end();
   }
 
   // ---- teardown: every thread of both CTAs gets here (all waits above are bounded) ----
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no remote store or arrival can target this CTA after this point
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)

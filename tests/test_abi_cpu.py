@@ -87,3 +87,30 @@ def test_null_cache_and_negative_n(hx):
     assert hx.lib.helix_attn_workspace_size(None, 128, ctypes.byref(n)) == 1
     assert hx.lib.helix_attn_workspace_size(ctypes.byref(s), 100, ctypes.byref(n)) == 1  # Hq % Hkv
     assert hx.lib.helix_attn_workspace_size(ctypes.byref(s), 256, ctypes.byref(n)) == 2  # G = 32
+
+
+def test_range_calls_reject_bad_ranges(hx):
+    buf = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    f = hx.lib.helix_attn_combine_range
+    assert f(2, 4, 8, 128, -1, 2, buf, buf, buf, 0, None, None) == 1  # negative begin
+    assert f(2, 4, 8, 128, 3, 2, buf, buf, buf, 0, None, None) == 1  # end < begin
+    assert f(2, 4, 8, 128, 0, 5, buf, buf, buf, 0, None, None) == 1  # end > batch
+    s = _struct(hx)
+    g = hx.lib.helix_attn_partial_range
+    assert g(ctypes.byref(s), buf, 128, 0.1, 0, 9, buf, buf, buf, 1 << 20, None) == 1
+    assert g(ctypes.byref(s), buf, 128, 0.1, 5, 4, buf, buf, buf, 1 << 20, None) == 1
+    assert g(None, buf, 128, 0.1, 0, 1, buf, buf, buf, 1 << 20, None) == 1
+
+
+def test_overlapped_rejects_missing_events_and_one_stream(hx):
+    s = _struct(hx)
+    buf = ctypes.c_void_p(16)
+    h = hx.lib.helix_attn_overlapped
+    ev = (ctypes.c_void_p * 3)(32, 64, 96)
+    args = lambda n, sa, sb, evs: (ctypes.byref(s), buf, 128, 0.1, n, buf, buf, buf, 0, None, buf,
+                                   1 << 20, sa, sb, evs)
+    assert h(*args(2, None, ctypes.c_void_p(8), None)) == 1  # no events
+    assert h(*args(2, ctypes.c_void_p(8), ctypes.c_void_p(8), ev)) == 1  # the same stream twice
+    assert h(*args(0, None, ctypes.c_void_p(8), ev)) == 1  # no groups
+    ev_null = (ctypes.c_void_p * 3)(32, None, 96)
+    assert h(*args(2, None, ctypes.c_void_p(8), ev_null)) == 1  # a null event handle

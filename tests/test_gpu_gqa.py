@@ -174,15 +174,27 @@ def test_gqa_repeat_variable_lengths_bit_identical(kv_dtype):
         _gpu.assert_close_lse(first[3][b, hs], L, f"LSE b={b}")
 
 
-def test_gqa_bad_page_id_sets_error_and_skips():
-    w = wl.WORKLOADS["gqa_s128k"].with_(B=1, Hq=16, Hkv=1, S=640, kvp=2)
+@pytest.mark.parametrize("kv_dtype", ["bf16", "nvfp4"])
+def test_gqa_bad_page_id_sets_error_and_skips(kv_dtype):
+    """A page id outside the pool sets the device error bit, and that page's 64 tokens are left out
+    of its shard; the rest of the shard is still attended exactly."""
+    base = wl.WORKLOADS["gqa_s128k" if kv_dtype == "bf16" else "gqa_nvfp4_s1m"]
+    w = base.with_(B=1, Hq=16, Hkv=1, S=640, kvp=2)
     cache = _gpu.make_cache(w)
     _gpu.fill(cache, w, [640])
-    cache.page_table[1, 0, 2] = 10 ** 6  # beyond the pool
+    cache.page_table[1, 0, 2] = 10 ** 6  # beyond the pool: local tokens 128..191 of shard 1
     cache.clear_errors()
     q = wl.query(w, "cuda")
-    _run(cache, w, q)
+    o_part, lse_part, _, _ = _run(cache, w, q)
     assert cache.err_bits() & _gpu.hx().DEVERR_PAGE_ID
+    K, V = _gpu.oracle_kv(w, 0, 0, 640)
+    qg = oracle.attention._f64(q[0, : w.G])
+    sets = _gpu.shard_sets(w, 640)
+    kept = np.concatenate([sets[1][:128], sets[1][192:]])
+    for s_, idx in ((0, sets[0]), (1, kept)):
+        Os, Ls = oracle.attend(qg, K[idx], V[idx], w.softmax_scale)
+        _gpu.assert_close_O(o_part[s_, 0, : w.G], Os, f"O_partial s={s_}")
+        _gpu.assert_close_lse(lse_part[s_, 0, : w.G], Ls, f"lse_partial s={s_}")
 
 
 # ---------------------------------------------------------------------------------------------
