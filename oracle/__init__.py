@@ -26,4 +26,4 @@ pages' round-robin example).  No function here is "parity unpinned".
 
 from .attention import attend, decode, partial, combine  # noqa: F401
 from .layout import rr_place, contig_place, shard_tokens, shard_lens, page_slot  # noqa: F401
-from .nvfp4 import e2m1_value, e4m3_value, nvfp4_dequant  # noqa: F401
+from .nvfp4 import e2m1_value, e4m3_value, nvfp4_dequant, nvfp4_encode  # noqa: F401

@@ -240,3 +240,45 @@ def pin_nvfp4(e2m1_value, e4m3_value, nvfp4_dequant):
     assert x.shape == (1, 32)
     assert x[0, 0] == 1.0 and x[0, 1] == 6.0 and x[0, 16] == -3.0 and x[0, 2] == 0.0
     assert x[0, 10] == 2.0 and x[0, 11] == 0.0 and x[0, 31] == 6.0 and x[0, 30] == 0.0
+
+
+def pin_nvfp4_encode(nvfp4_encode, seed=6):
+    """The quantiser: hand-derived blocks (every E2M1 tie, saturation, the 448 clamp, scale 0,
+    a subnormal scale, E4M3 scale ties), the scale against torch's float8_e4m3fn rounding, the
+    per-element error bound, and agreement with the input generator's separate encoder."""
+    for name, vals, sc, codes in (
+            [p.strip() for p in " ".join(r).split("|")] for r in _golden_rows("nvfp4_encode_cases.txt")):
+        x = np.array([float(v) for v in vals.split()], dtype=np.float32)[None]
+        c, s = nvfp4_encode(x)
+        assert int(np.asarray(s)[0, 0]) == int(sc, 16), f"{name}: scale"
+        assert [int(v) for v in np.asarray(c)[0]] == [int(b, 16) for b in codes.split()], name
+    g = torch.Generator().manual_seed(seed)
+    # magnitudes over many binades, including blocks whose absmax / 6 exceeds 448 or underflows
+    x = torch.randn(512, 64, generator=g) * torch.exp2(torch.randint(-14, 13, (512, 1), generator=g).float())
+    x[0] = 0.0
+    c, s = nvfp4_encode(x)
+    c, s = np.asarray(c), np.asarray(s)
+    amax = x.reshape(512, 4, 16).abs().amax(-1)
+    r = (amax / 6.0).clamp(max=448.0).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(s, r), "scale differs from torch's E4M3 rounding"
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    half_gap = np.array([0.25, 0.25, 0.25, 0.25, 0.5, 0.5, 1.0, 1.0])  # max error per magnitude
+    lo = c & 0xF
+    hi = c >> 4
+    code = np.stack([lo, hi], -1).reshape(512, 64)
+    sign = np.where(code & 8, -1.0, 1.0)
+    mag_i = code & 7
+    sd = np.repeat(torch.from_numpy(s.copy()).view(torch.float8_e4m3fn).double().numpy(), 16,
+                   axis=1)
+    xd = x.double().numpy()
+    y = np.where(sd > 0, xd / np.where(sd > 0, sd, 1.0), xd)
+    dec = sign * mags[mag_i]
+    sat = np.abs(y) > 6.0
+    assert np.all(np.abs(dec[~sat] - y[~sat]) <= half_gap[mag_i][~sat] * (1 + 1e-6) + 1e-12)
+    assert np.all(np.abs(dec[sat]) == 6.0) and np.all(np.sign(dec[sat]) == np.sign(y[sat]))
+    assert not np.any((mag_i == 0) & (code & 8)), "a zero magnitude carries a sign"
+    # an independent encoder (the input generator's, thresholds in torch) gives the same bytes
+    import workloads
+
+    c2, s2 = workloads.nvfp4_encode(x)
+    assert np.array_equal(c, c2.numpy()) and np.array_equal(s, s2.numpy())

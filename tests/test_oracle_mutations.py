@@ -166,9 +166,73 @@ def test_nvfp4_mutants_caught(which):
     assert _caught(_pins.pin_nvfp4, e2, e4, dq)
 
 
+def _enc_ties_away(x):
+    saved = N4._nearest_even
+
+    def away(a, table):
+        d = np.abs(np.asarray(a, float)[..., None] - table)
+        dmin = d.min(-1, keepdims=True)
+        idx = np.arange(table.shape[0])
+        return np.where(d == dmin, idx, -1).max(-1)  # larger entry on a tie
+    N4._nearest_even = away
+    try:
+        return N4.nvfp4_encode(x)
+    finally:
+        N4._nearest_even = saved
+
+
+def _enc_truncate(x):
+    saved = N4._nearest_even
+
+    def floor_(a, table):
+        a = np.asarray(a, float)
+        return (a[..., None] >= table).sum(-1) - 1
+    N4._nearest_even = floor_
+    try:
+        return N4.nvfp4_encode(x)
+    finally:
+        N4._nearest_even = saved
+
+
+def _enc_signed_max(x):
+    x = np.asarray(x, np.float32)
+    c, s = N4.nvfp4_encode(x)
+    xb = x.reshape(*x.shape[:-1], -1, 16)
+    r = (np.maximum(xb.max(-1), 0) / np.float32(6)).astype(np.float32)
+    return c, N4.e4m3_encode_satfinite(r)
+
+
+def _enc_no_clamp(x):
+    x = np.asarray(x, np.float32)
+    c, s = N4.nvfp4_encode(x)
+    big = np.abs(x.reshape(*x.shape[:-1], -1, 16)).max(-1) / 6 > 448
+    return c, np.where(big, np.uint8(0x7F), s)  # overflow to NaN instead of 448
+
+
+def _enc_negative_zero(x):
+    x = np.asarray(x, np.float32)
+    c, s = N4.nvfp4_encode(x)
+    neg = (x < 0).reshape(*x.shape[:-1], -1, 2)
+    lo = np.where(((c & 0xF) == 0) & neg[..., 0], c | 0x8, c)
+    return np.where(((lo >> 4) == 0) & neg[..., 1], lo | 0x80, lo).astype(np.uint8), s
+
+
+def _enc_swapped_nibbles(x):
+    c, s = N4.nvfp4_encode(x)
+    return ((c & 0xF) << 4 | (c >> 4)).astype(np.uint8), s
+
+
+@pytest.mark.parametrize("mut", [_enc_ties_away, _enc_truncate, _enc_signed_max, _enc_no_clamp,
+                                 _enc_negative_zero, _enc_swapped_nibbles],
+                         ids=lambda f: f.__name__)
+def test_nvfp4_encode_mutants_caught(mut):
+    assert _caught(_pins.pin_nvfp4_encode, mut)
+
+
 def test_real_oracle_passes_every_pin():
     _pins.pin_brute_force(oracle.attend)
     _pins.pin_closed_forms(oracle.attend)
     _pins.pin_invariances(oracle.attend)
     _pins.pin_torch_sdpa(oracle.decode)
     _pins.pin_combine_identity(oracle.attend, oracle.combine, oracle.shard_tokens)
+    _pins.pin_nvfp4_encode(oracle.nvfp4_encode)

@@ -82,3 +82,7 @@ def test_workload_bytes_positive(name):
     lens = wl.seq_lens(w)
     assert all(1 <= s <= w.S for s in lens)
     assert wl.step_bytes(w, lens) > wl.partial_bytes(w, lens) > 0
+
+
+def test_nvfp4_encode():
+    _pins.pin_nvfp4_encode(oracle.nvfp4_encode)
