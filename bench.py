@@ -291,8 +291,23 @@ def run_helix(args):
     torch.cuda.synchronize()
     assert cache.err_bits() == 0, "prefill reported a device error"
     # the new token of every step, resident as [step][B][1][...] so each step's slice is dense
-    step_rows = {k: v.transpose(0, 1).unsqueeze(2).contiguous()
-                 for k, v in wl.append_rows(w, 0, n_steps, dev).items()}
+    # An NVFP4 cache takes the new token as bf16 rows and encodes it on the device
+    # (helix_kv_append_quantize), as a decode loop over an FP4 cache does.
+    quant = w.kv_dtype == "nvfp4"
+    if quant:
+        new_rows = {"k_new": torch.stack([wl.kv_tokens(w, "k", b, 0, n_steps, dev)
+                                          for b in range(w.B)]),
+                    "v_new": torch.stack([wl.kv_tokens(w, "v", b, 0, n_steps, dev)
+                                          for b in range(w.B)])}
+    else:
+        new_rows = wl.append_rows(w, 0, n_steps, dev)
+    step_rows = {k: v.transpose(0, 1).unsqueeze(2).contiguous() for k, v in new_rows.items()}
+
+    def append_step(a):
+        if quant:
+            hx.append_quantize(cache, a["k_new"], a["v_new"])
+        else:
+            hx.append(cache, a["k_new"], a.get("v_new"), a.get("k_scale"), a.get("v_scale"))
     q = wl.query(w, dev)
     o_part = torch.empty(w.kvp, w.B, w.Hq, w.dv, dtype=torch.float32, device=dev)
     lse_part = torch.empty(w.kvp, w.B, w.Hq, dtype=torch.float32, device=dev)
@@ -302,8 +317,7 @@ def run_helix(args):
     stream = torch.cuda.current_stream()
 
     def one_step(i, ev=None):
-        a = {k: v[i] for k, v in step_rows.items()}
-        hx.append(cache, a["k_new"], a.get("v_new"), a.get("k_scale"), a.get("v_scale"))
+        append_step({k: v[i] for k, v in step_rows.items()})
         if ev is not None:
             ev[0].record(stream)
         hx.partial(cache, q, w.softmax_scale, o_part, lse_part, ws)
@@ -360,8 +374,7 @@ def run_helix(args):
             q_d.copy_(q_h, non_blocking=True)
             for k_ in tok_d:
                 tok_d[k_].copy_(rows_h[k_][si + i], non_blocking=True)
-            hx.append(cache, tok_d["k_new"], tok_d.get("v_new"), tok_d.get("k_scale"),
-                      tok_d.get("v_scale"))
+            append_step(tok_d)
             hx.partial(cache, q_d, w.softmax_scale, o_part, lse_part, ws)
             hx.combine(o_part, lse_part, out, lse_out)
             out_h.copy_(out, non_blocking=True)
@@ -380,8 +393,7 @@ def run_helix(args):
         ov = hx.Overlap(args.hopb_groups, dev)
 
         def hopb_step(i):
-            a = {k: v[i] for k, v in step_rows.items()}
-            hx.append(cache, a["k_new"], a.get("v_new"), a.get("k_scale"), a.get("v_scale"))
+            append_step({k: v[i] for k, v in step_rows.items()})
             hx.overlapped(cache, q, w.softmax_scale, ov, o_part, lse_part, out, lse_out,
                           workspace=ws)
 
@@ -413,7 +425,8 @@ def run_helix(args):
         peak, tflops_peak, peak_kind = measured_peaks()
         achieved_gbs = part_bytes / (part_ms * 1e-3) / 1e9
         kname = ("mla_partial_kernel" if w.kind == "mla" else
-                 f"gqa_partial_kernel<{w.d},{w.kv_dtype}>")
+                 "gqa_partial_nvfp4_kernel" if w.kv_dtype == "nvfp4" else
+                 f"gqa_partial_kernel<{w.d}>")
         flops = float(np.mean([wl.partial_flops(w, L) for L in lens_at]))
         achieved_tf = flops / (part_ms * 1e-3) / 1e12
         hbm = {"achieved": achieved_gbs, "peak": peak, "unit": "GB/s", "frac": achieved_gbs / peak}

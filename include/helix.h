@@ -131,6 +131,20 @@ helix_status helix_kv_append(const helix_kv_cache* cache, const void* k_new, con
                              const int32_t* n_valid, helix_stream_t stream);
 
 /*
+ * helix_kv_append for an NVFP4 GQA cache (head_dim 128) from bf16 rows, encoding on the device:
+ *   k_new, v_new bf16 [B][n_new][H][128] (16-byte aligned); n_valid as in helix_kv_append.
+ * Each 16-element block of a row gets scale = the E4M3 value nearest to fp32(absmax / 6) (ties to
+ * even, clamped to 448) and codes = the E2M1 values nearest to fp32(x / scale) (x itself when the
+ * scale is 0; ties to even, saturating at 6; a value rounding to zero is stored as +0), every
+ * division in IEEE fp32. The pages say only "FP4"; the block size, scale type and absmax / 6 rule
+ * are those of the NVFP4 format. Placement, lengths and device errors as helix_kv_append.
+ * Returns HELIX_ERR_UNSUPPORTED for other cache kinds.
+ */
+helix_status helix_kv_append_quantize(const helix_kv_cache* cache, const void* k_new,
+                                      const void* v_new, int32_t n_new, const int32_t* n_valid,
+                                      helix_stream_t stream);
+
+/*
  * Bytes of workspace helix_attn_partial needs for this cache shape on the current device.
  * The workspace must be zero-filled once before its first use; the kernel returns it to that
  * state, so later calls need no clearing (unless a previous call was aborted by a device error).

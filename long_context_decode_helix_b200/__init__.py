@@ -56,6 +56,8 @@ def _load():
     cache_p = ctypes.POINTER(CacheStruct)
     lib.helix_kv_append.argtypes = [cache_p, P, P, P, P, I32, P, P]
     lib.helix_kv_append.restype = I32
+    lib.helix_kv_append_quantize.argtypes = [cache_p, P, P, I32, P, P]
+    lib.helix_kv_append_quantize.restype = I32
     lib.helix_attn_workspace_size.argtypes = [cache_p, I32, ctypes.POINTER(SZ)]
     lib.helix_attn_workspace_size.restype = I32
     lib.helix_attn_partial.argtypes = [cache_p, P, I32, F32, P, P, P, SZ, P]
@@ -190,6 +192,15 @@ def append(cache: KVCache, k_new, v_new=None, k_scale=None, v_scale=None, n_vali
     _check(lib.helix_kv_append(ctypes.byref(cache.struct), _ptr(k_new), _ptr(v_new),
                                _ptr(k_scale), _ptr(v_scale), n_new, _ptr(n_valid),
                                _stream(stream)), "helix_kv_append")
+
+
+def append_quantize(cache: KVCache, k_new, v_new, n_valid=None, stream=None):
+    """Append bf16 rows [B, n_new, Hkv, 128] to an NVFP4 cache, encoding them on the device
+    (``helix_kv_append_quantize``)."""
+    n_new = int(k_new.shape[1])
+    _check(lib.helix_kv_append_quantize(ctypes.byref(cache.struct), _ptr(k_new), _ptr(v_new),
+                                        n_new, _ptr(n_valid), _stream(stream)),
+           "helix_kv_append_quantize")
 
 
 def workspace_size(cache: KVCache, num_q_heads: int) -> int:

@@ -220,6 +220,43 @@ helix_status helix_kv_append(const helix_kv_cache* c, const void* k_new, const v
   return append_launch(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+helix_status helix_kv_append_quantize(const helix_kv_cache* c, const void* k_new,
+                                      const void* v_new, int32_t n_new, const int32_t* n_valid,
+                                      helix_stream_t stream) {
+  helix_status st = check_cache(c);
+  if (st != HELIX_OK) return st;
+  if (c->kind != HELIX_ATTN_GQA || c->kv_dtype != HELIX_KV_NVFP4) return HELIX_ERR_UNSUPPORTED;
+  if (c->head_dim != 128 || c->page_tokens % 2 != 0) return HELIX_ERR_UNSUPPORTED;
+  if (n_new < 0) return HELIX_ERR_INVALID_ARG;
+  if (n_new == 0) return HELIX_OK;
+  if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new) ||
+      !aligned4(n_valid))
+    return HELIX_ERR_INVALID_ARG;
+  AppendParams p{};
+  p.src[0] = (const uint8_t*)k_new; p.dst[0] = (uint8_t*)c->k_pool; p.row_bytes[0] = 256;
+  p.src[1] = (const uint8_t*)v_new; p.dst[1] = (uint8_t*)c->v_pool; p.row_bytes[1] = 256;
+  p.dst[2] = (uint8_t*)c->k_scale;
+  p.dst[3] = (uint8_t*)c->v_scale;
+  p.quantize = 1;
+  p.v_nvfp4 = 1;
+  p.page_table = c->page_table;
+  p.shard_lens = c->shard_lens;
+  p.seq_lens = c->seq_lens;
+  p.err = c->err_word;
+  p.B = c->batch;
+  p.Hkv = c->num_kv_heads;
+  p.kvp = c->kvp;
+  p.layout = c->layout;
+  p.rr_block = c->rr_block;
+  p.contig_chunk = c->contig_chunk;
+  p.page_tokens = c->page_tokens;
+  p.max_pages = c->max_pages_per_shard;
+  p.num_pages = c->num_pages;
+  p.n_new = n_new;
+  p.n_valid = n_valid;
+  return append_launch(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 helix_status helix_attn_workspace_size(const helix_kv_cache* c, int32_t num_q_heads,
                                        size_t* bytes) {
   if (bytes == nullptr) return HELIX_ERR_INVALID_ARG;

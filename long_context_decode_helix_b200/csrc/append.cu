@@ -10,6 +10,7 @@
 // The copy is bit-exact (16/8/4-byte vector moves). Lengths advance after every copy of the call has
 // read the old seq_lens: in the same block when one block holds all of a request's new tokens,
 // otherwise in a second one-block kernel on the same stream.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -72,6 +73,58 @@ __device__ void copy_bytes(uint8_t* dst, const uint8_t* src, int bytes, int lane
   else copy_row<4>(dst, src, bytes, lane0, nlanes);
 }
 
+// ---- on-device NVFP4 encoding of one bf16 row of 128 elements (one warp; lane l holds elements
+// 4l .. 4l+3, so lanes 4k .. 4k+3 hold scale block k). Every rounding decision is taken in fp32:
+// scale = E4M3(fp32(absmax / 6)) rounded to nearest even and clamped to 448 (satfinite);
+// code = E2M1(fp32(x / scale)) rounded to nearest even, saturating at 6 (x itself when the scale is
+// 0); a code whose magnitude rounds to zero is stored as +0.
+struct Nvfp4Lane {
+  uint32_t codes16;  // 4 codes, element 4l + e in bits [4e, 4e + 4)
+  uint32_t scale;    // E4M3 byte of this lane's block
+};
+
+__device__ __forceinline__ uint32_t e4m3_rn_satfinite(float r) {
+  uint16_t v;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(v) : "f"(0.f), "f"(r));
+  return v & 0xFFu;  // the second source lands in the low byte
+}
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)byte));
+  return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
+}
+// two codes in one byte: lo in bits 0-3, hi in bits 4-7
+__device__ __forceinline__ uint32_t e2m1x2_rn_satfinite(float lo, float hi) {
+  uint16_t v;
+  asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u16.u8 %0, t;\n}"
+      : "=h"(v) : "f"(hi), "f"(lo));
+  uint32_t b = v & 0xFFu;
+  if ((b & 0x07u) == 0) b &= 0xF0u;  // -0 -> +0
+  if ((b & 0x70u) == 0) b &= 0x0Fu;
+  return b;
+}
+
+__device__ __forceinline__ Nvfp4Lane encode_lane(const uint8_t* row_bf16, int lane) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(row_bf16 + 8 * lane);
+  const float x0 = __uint_as_float(raw.x << 16), x1 = __uint_as_float(raw.x & 0xFFFF0000u);
+  const float x2 = __uint_as_float(raw.y << 16), x3 = __uint_as_float(raw.y & 0xFFFF0000u);
+  float a = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  Nvfp4Lane r;
+  r.scale = e4m3_rn_satfinite(__fdiv_rn(a, 6.f));
+  const float sd = e4m3_to_f32(r.scale);
+  float y0 = x0, y1 = x1, y2 = x2, y3 = x3;
+  if (sd > 0.f) {
+    y0 = __fdiv_rn(x0, sd);
+    y1 = __fdiv_rn(x1, sd);
+    y2 = __fdiv_rn(x2, sd);
+    y3 = __fdiv_rn(x3, sd);
+  }
+  r.codes16 = e2m1x2_rn_satfinite(y0, y1) | (e2m1x2_rn_satfinite(y2, y3) << 8);
+  return r;
+}
+
 __device__ __forceinline__ int rows_of(const AppendParams& p, int b) {
   if (p.n_valid == nullptr) return p.n_new;
   return min(max(p.n_valid[b], 0), p.n_new);
@@ -119,7 +172,27 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
     }
     const size_t src_row = ((size_t)b * p.n_new + j) * p.Hkv + h;
     const size_t dst_row = ((size_t)page * p.Hkv + h) * p.page_tokens + slot;
-    if (!p.v_nvfp4) {
+    if (p.quantize) {
+      // d = 128: K codes row of 64 bytes (lane l: bytes 2l, 2l+1), 8 scale bytes, V codes into the
+      // token-pair layout (lane l: column word l), V scales block-major
+      const Nvfp4Lane k = encode_lane(p.src[0] + src_row * 256, lane);
+      const Nvfp4Lane v = encode_lane(p.src[1] + src_row * 256, lane);
+      *reinterpret_cast<uint16_t*>(p.dst[0] + dst_row * 64 + 2 * lane) = (uint16_t)k.codes16;
+      if ((lane & 3) == 0) p.dst[2][dst_row * 8 + (lane >> 2)] = (uint8_t)k.scale;
+      const int pair = slot / 2, shift = 4 * (slot & 1);
+      uint32_t* vblk = reinterpret_cast<uint32_t*>(
+          p.dst[1] + (((size_t)page * p.Hkv + h) * (p.page_tokens / 2) + pair) * 128);
+      uint32_t bits = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) bits |= ((v.codes16 >> (4 * e)) & 0xFu) << (8 * e + shift);
+      const int wd = lane;  // columns 4 wd .. 4 wd + 3
+      const int sw = ((((wd >> 2) ^ ((pair & 3) << 1))) << 2) | (wd & 3);
+      atomicAnd(vblk + sw, ~(0x0F0F0F0Fu << shift));
+      atomicOr(vblk + sw, bits);
+      if ((lane & 3) == 0)
+        p.dst[3][(((size_t)page * p.Hkv + h) * 8 + (lane >> 2)) * p.page_tokens + slot] =
+            (uint8_t)v.scale;
+    } else if (!p.v_nvfp4) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int rb = p.row_bytes[k];

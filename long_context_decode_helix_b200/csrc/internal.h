@@ -67,6 +67,8 @@ struct AppendParams {
   uint32_t* err;
   const int32_t* n_valid;  // optional [B]
   int v_nvfp4;             // 1: streams 1 and 3 (V codes, V scales) use the token-pair layout
+  int quantize;            // 1: src[0] / src[1] are bf16 K / V rows of d = 128, encoded to NVFP4
+                           //    on the device into the four NVFP4 pools (dst[0..3])
   int B, Hkv, kvp, layout, rr_block, contig_chunk, page_tokens, max_pages, num_pages, n_new;
 };
 helix_status append_launch(const AppendParams& p, cudaStream_t stream);
