@@ -12,9 +12,9 @@
 // Why its own kernel: at 4.5 bits per element the cache streams four times faster than bf16, and
 // every element has to be decoded in registers (a cvt of two codes and an f16x2 multiply by their
 // scale per pair), so the per-token instruction count, not HBM, bounds a kernel that spreads a page
-// over four warps. Here one warp owns a whole 64-token page: 8 consumer warps work on 8 different
-// pages, every page-level step (row max, rescale decision, shuffles) is amortised over 64 tokens,
-// and the four n-tiles of a 32-token half give four independent MMA chains.
+// over four warps. Here one warp owns a whole 64-token page: 8 warps work on 8 different pages,
+// every page-level step (row max, rescale decision, shuffles) is amortised over 64 tokens, and the
+// eight n-tiles of the page give eight independent MMA chains for S.
 //
 // Per page and warp (16 head rows = the M of an m16n8k16 tile, f16 in, fp32 accumulate):
 //   S = q K^T: a lane reads 16 code bytes (32 elements) of one token per n-tile; the MMA's k index
@@ -278,19 +278,18 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
   bool dead = false;
   const float sl2 = p.scale_log2;
 
-  // One page (64 tokens, nvalid of them in the history) from ring stage st.
+  // One page (64 tokens, nvalid of them in the history) from ring stage st, all at once: eight
+  // n-tiles of S (eight independent MMA chains), one softmax pass and one rescale decision for the
+  // page, then P V over four 16-token k-chunks.
   auto process_page = [&](const uint8_t* st, int nvalid) {
-    const bool full = nvalid >= kPage;
+    // ---- S = q K^T: n-tile n holds tokens 8 n + (0..7); this lane's token of n-tile n is 8n + g8
+    float s[8][4];
+    {
+      uint4 kc[8];
+      uint32_t sc2[8];  // (scale of elements [32 t, 32 t + 16), of [32 t + 16, 32 t + 32))
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      if (32 * hh >= nvalid) break;
-      // ---- S = q K^T for tokens [32 hh, 32 hh + 32): n-tile n holds tokens 32 hh + 8 n + (0..7)
-      float s[4][4];
-      uint4 kc[4];
-      uint32_t sc2[4];  // (scale of elements [32 t, 32 t + 16), of [32 t + 16, 32 t + 32))
-#pragma unroll
-      for (int n = 0; n < 4; ++n) {
-        const int token = 32 * hh + 8 * n + g8;
+      for (int n = 0; n < 8; ++n) {
+        const int token = 8 * n + g8;
         kc[n] = *reinterpret_cast<const uint4*>(st + token * (kD / 2) + t4 * 16);
         sc2[n] =
             e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(st + kOffKs + token * 8 + 2 * t4));
@@ -299,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
 #pragma unroll
       for (int wq = 0; wq < 4; ++wq) {  // code word wq holds k-steps 2 wq and 2 wq + 1
 #pragma unroll
-        for (int n = 0; n < 4; ++n) {
+        for (int n = 0; n < 8; ++n) {
           const uint32_t word = wq == 0 ? kc[n].x : wq == 1 ? kc[n].y : wq == 2 ? kc[n].z : kc[n].w;
           uint32_t h0, h1, h2, h3;
           e2m1x4_to_f16x2(word, h0, h1, h2, h3);
@@ -312,86 +311,86 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
           }
         }
       }
-      // ---- online softmax over the half (base 2, lazy reference maximum)
-      float x[4][4];
+    }
+    // ---- online softmax over the page (base 2, lazy reference maximum)
 #pragma unroll
-      for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < 8; ++n)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[n][e] = s[n][e] * sl2;
-      if (!full) {
+      for (int e = 0; e < 4; ++e) s[n][e] *= sl2;
+    if (nvalid < kPage) {
 #pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          const int t = 32 * hh + 8 * n + 2 * t4;
-          if (t >= nvalid) x[n][0] = x[n][2] = -INFINITY;
-          if (t + 1 >= nvalid) x[n][1] = x[n][3] = -INFINITY;
-        }
+      for (int n = 0; n < 8; ++n) {
+        const int t = 8 * n + 2 * t4;
+        if (t >= nvalid) s[n][0] = s[n][2] = -INFINITY;
+        if (t + 1 >= nvalid) s[n][1] = s[n][3] = -INFINITY;
       }
-      float mx0 = fmaxf(fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1])),
-                        fmaxf(fmaxf(x[2][0], x[2][1]), fmaxf(x[3][0], x[3][1])));
-      float mx1 = fmaxf(fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3])),
-                        fmaxf(fmaxf(x[2][2], x[2][3]), fmaxf(x[3][2], x[3][3])));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const bool up0 = mx0 > m_ref[0] + kLazy, up1 = mx1 > m_ref[1] + kLazy;
-      if (__any_sync(0xffffffffu, up0 || up1)) {
-        const float n0 = up0 ? mx0 : m_ref[0], n1 = up1 ? mx1 : m_ref[1];
-        const float a0 = up0 ? fast_exp2(m_ref[0] - n0) : 1.f;  // exp2(-inf) = 0 at the start
-        const float a1 = up1 ? fast_exp2(m_ref[1] - n1) : 1.f;
-        m_ref[0] = n0;
-        m_ref[1] = n1;
+    }
+    float mx0 = fmaxf(s[0][0], s[0][1]), mx1 = fmaxf(s[0][2], s[0][3]);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          O[j][0] *= a0;
-          O[j][1] *= a0;
-          O[j][2] *= a1;
-          O[j][3] *= a1;
-        }
-        lb[0] *= a0;
-        lb[1] *= a0;
-        lb[2] *= a1;
-        lb[3] *= a1;
+    for (int n = 1; n < 8; ++n) {
+      mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
+      mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const bool up0 = mx0 > m_ref[0] + kLazy, up1 = mx1 > m_ref[1] + kLazy;
+    if (__any_sync(0xffffffffu, up0 || up1)) {
+      const float n0 = up0 ? mx0 : m_ref[0], n1 = up1 ? mx1 : m_ref[1];
+      const float a0 = up0 ? fast_exp2(m_ref[0] - n0) : 1.f;  // exp2(-inf) = 0 at the start
+      const float a1 = up1 ? fast_exp2(m_ref[1] - n1) : 1.f;
+      m_ref[0] = n0;
+      m_ref[1] = n1;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        O[j][0] *= a0;
+        O[j][1] *= a0;
+        O[j][2] *= a1;
+        O[j][3] *= a1;
       }
-      const float mu0 = m_ref[0] == -INFINITY ? 0.f : m_ref[0];
-      const float mu1 = m_ref[1] == -INFINITY ? 0.f : m_ref[1];
-      // ---- O += P V, one 16-token k-chunk at a time
+      lb[0] *= a0;
+      lb[1] *= a0;
+      lb[2] *= a1;
+      lb[3] *= a1;
+    }
+    const float mu0 = m_ref[0] == -INFINITY ? 0.f : m_ref[0];
+    const float mu1 = m_ref[1] == -INFINITY ? 0.f : m_ref[1];
+    // ---- O += P V, one 16-token k-chunk (n-tiles 2 cc, 2 cc + 1) at a time
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int cc = 2 * hh + c;  // k-chunk of the page: tokens [16 cc, 16 cc + 16)
-        uint32_t pa[4];
-        pa[0] = pack_f16x2(fast_exp2(x[2 * c][0] - mu0), fast_exp2(x[2 * c][1] - mu0));
-        pa[1] = pack_f16x2(fast_exp2(x[2 * c][2] - mu1), fast_exp2(x[2 * c][3] - mu1));
-        pa[2] = pack_f16x2(fast_exp2(x[2 * c + 1][0] - mu0), fast_exp2(x[2 * c + 1][1] - mu0));
-        pa[3] = pack_f16x2(fast_exp2(x[2 * c + 1][2] - mu1), fast_exp2(x[2 * c + 1][3] - mu1));
-        // token pairs (2t, 2t+1) and (2t+8, 2t+9) of the chunk; a pair row's 16-byte chunks are
-        // stored XOR-swizzled by 2 (pair mod 4) = 2t, so a quarter-warp hits every bank once
-        const int pa_ = 8 * cc + t4, pb_ = pa_ + 4;
-        const int sw = (g8 ^ (t4 << 1)) << 4;
-        const uint4 va = *reinterpret_cast<const uint4*>(st + kOffVc + pa_ * kD + sw);
-        const uint4 vb = *reinterpret_cast<const uint4*>(st + kOffVc + pb_ * kD + sw);
-        const uint8_t* vsc = st + kOffVs + g8 * kPage + 16 * cc + 2 * t4;
-        uint32_t sa = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc));
-        uint32_t sb = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc + 8));
-        if (!full) {  // tokens past the history: zero scale, so their codes contribute nothing
-          const int ta = 16 * cc + 2 * t4, tb = ta + 8;
-          sa &= (ta < nvalid ? 0x0000ffffu : 0u) | (ta + 1 < nvalid ? 0xffff0000u : 0u);
-          sb &= (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
-        }
-        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (int wq = 0; wq < 4; ++wq) {
-          uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-          e2m1x4_to_f16x2(wa[wq], a0, a1, a2, a3);
-          e2m1x4_to_f16x2(wb[wq], c0, c1, c2, c3);
-          mma_f16_16816(O[4 * wq + 0], pa, hmul2(a0, sa), hmul2(c0, sb));
-          mma_f16_16816(O[4 * wq + 1], pa, hmul2(a1, sa), hmul2(c1, sb));
-          mma_f16_16816(O[4 * wq + 2], pa, hmul2(a2, sa), hmul2(c2, sb));
-          mma_f16_16816(O[4 * wq + 3], pa, hmul2(a3, sa), hmul2(c3, sb));
-        }
-        mma_f16_16816(lb, pa, kOnes, kOnes);
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t pa[4];
+      pa[0] = pack_f16x2(fast_exp2(s[2 * cc][0] - mu0), fast_exp2(s[2 * cc][1] - mu0));
+      pa[1] = pack_f16x2(fast_exp2(s[2 * cc][2] - mu1), fast_exp2(s[2 * cc][3] - mu1));
+      pa[2] = pack_f16x2(fast_exp2(s[2 * cc + 1][0] - mu0), fast_exp2(s[2 * cc + 1][1] - mu0));
+      pa[3] = pack_f16x2(fast_exp2(s[2 * cc + 1][2] - mu1), fast_exp2(s[2 * cc + 1][3] - mu1));
+      // token pairs (2t, 2t+1) and (2t+8, 2t+9) of the chunk; a pair row's 16-byte chunks are
+      // stored XOR-swizzled by 2 (pair mod 4) = 2t, so a quarter-warp hits every bank once
+      const int pa_ = 8 * cc + t4, pb_ = pa_ + 4;
+      const int sw = (g8 ^ (t4 << 1)) << 4;
+      const uint4 va = *reinterpret_cast<const uint4*>(st + kOffVc + pa_ * kD + sw);
+      const uint4 vb = *reinterpret_cast<const uint4*>(st + kOffVc + pb_ * kD + sw);
+      const uint8_t* vsc = st + kOffVs + g8 * kPage + 16 * cc + 2 * t4;
+      uint32_t sa = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc));
+      uint32_t sb = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(vsc + 8));
+      if (nvalid < kPage) {  // tokens past the history: zero scale, so their codes contribute nothing
+        const int ta = 16 * cc + 2 * t4, tb = ta + 8;
+        sa &= (ta < nvalid ? 0x0000ffffu : 0u) | (ta + 1 < nvalid ? 0xffff0000u : 0u);
+        sb &= (tb < nvalid ? 0x0000ffffu : 0u) | (tb + 1 < nvalid ? 0xffff0000u : 0u);
       }
+      const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+      const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+      for (int wq = 0; wq < 4; ++wq) {
+        uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+        e2m1x4_to_f16x2(wa[wq], a0, a1, a2, a3);
+        e2m1x4_to_f16x2(wb[wq], c0, c1, c2, c3);
+        mma_f16_16816(O[4 * wq + 0], pa, hmul2(a0, sa), hmul2(c0, sb));
+        mma_f16_16816(O[4 * wq + 1], pa, hmul2(a1, sa), hmul2(c1, sb));
+        mma_f16_16816(O[4 * wq + 2], pa, hmul2(a2, sa), hmul2(c2, sb));
+        mma_f16_16816(O[4 * wq + 3], pa, hmul2(a3, sa), hmul2(c3, sb));
+      }
+      mma_f16_16816(lb, pa, kOnes, kOnes);
     }
   };
 
