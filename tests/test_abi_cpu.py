@@ -114,3 +114,9 @@ def test_overlapped_rejects_missing_events_and_one_stream(hx):
     assert h(*args(0, None, ctypes.c_void_p(8), ev)) == 1  # no groups
     ev_null = (ctypes.c_void_p * 3)(32, None, 96)
     assert h(*args(2, None, ctypes.c_void_p(8), ev_null)) == 1  # a null event handle
+
+
+def test_partial_combine_rejects_a_missing_cache(hx):
+    buf = ctypes.c_void_p(16)
+    f = hx.lib.helix_attn_partial_combine
+    assert f(None, buf, 128, 0.1, buf, buf, buf, 0, None, buf, 1 << 20, None) == 1
