@@ -273,6 +273,8 @@ def run_helix(args):
     K, W = args.steps, args.warmup
     n_steps = K + W + (K if not args.no_e2e else 0) + (W + K if args.hopb_groups > 0 else 0)
     S_cap = max(lens) + n_steps + 16
+    if w.layout == "contig":  # size the contiguous shards for the history plus the new tokens
+        w = w.with_(S_final=S_cap)
 
     # --- state resident in HBM: the history (S_b - 1 tokens), then one new token per step ---
     pt, n_pages = wl.page_table(w, S_cap)
@@ -320,10 +322,10 @@ def run_helix(args):
         append_step({k: v[i] for k, v in step_rows.items()})
         if ev is not None:
             ev[0].record(stream)
-        hx.partial(cache, q, w.softmax_scale, o_part, lse_part, ws)
+        # partial attention and the combine: one launch for GQA (helix_attn_partial_combine)
+        hx.partial_combine(cache, q, w.softmax_scale, o_part, lse_part, out, lse_out, workspace=ws)
         if ev is not None:
             ev[1].record(stream)
-        hx.combine(o_part, lse_part, out, lse_out)
 
     si = 0
     for _ in range(W):
@@ -375,8 +377,8 @@ def run_helix(args):
             for k_ in tok_d:
                 tok_d[k_].copy_(rows_h[k_][si + i], non_blocking=True)
             append_step(tok_d)
-            hx.partial(cache, q_d, w.softmax_scale, o_part, lse_part, ws)
-            hx.combine(o_part, lse_part, out, lse_out)
+            hx.partial_combine(cache, q_d, w.softmax_scale, o_part, lse_part, out, lse_out,
+                               workspace=ws)
             out_h.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -393,9 +395,15 @@ def run_helix(args):
         ov = hx.Overlap(args.hopb_groups, dev)
 
         def hopb_step(i):
-            append_step({k: v[i] for k, v in step_rows.items()})
-            hx.overlapped(cache, q, w.softmax_scale, ov, o_part, lse_part, out, lse_out,
-                          workspace=ws)
+            a = {k: v[i] for k, v in step_rows.items()}
+            if quant:  # the device-encoding append is not part of the overlapped call
+                append_step(a)
+                hx.overlapped(cache, q, w.softmax_scale, ov, o_part, lse_part, out, lse_out,
+                              workspace=ws)
+            else:  # append, partial and combine of request groups over two streams
+                hx.decode_overlapped(cache, q, w.softmax_scale, ov, a["k_new"], a.get("v_new"),
+                                     o_partial=o_part, lse=lse_part, out=out, lse_out=lse_out,
+                                     workspace=ws)
 
         for _ in range(W):
             hopb_step(si)
@@ -415,18 +423,19 @@ def run_helix(args):
         per = -(-w.B // n_groups)
         hopb = {"groups": -(-w.B // per), "us_per_step": hopb_ms * 1e3,
                 "serial_us_per_step": ms_step * 1e3, "speedup": ms_step / hopb_ms,
-                "gpu_launches": K * (1 + 2 * (-(-w.B // per)))}
+                "gpu_launches": K * 3 * (-(-w.B // per))}
         assert cache.err_bits() == 0, "a HOP-B step reported a device error"
 
     if rank == 0:
         step_bytes = float(np.mean([wl.step_bytes(w, L) for L in lens_at]))
-        part_bytes = float(np.mean([wl.partial_bytes(w, L) for L in lens_at]))
+        # the timed kernel: the fused partial + combine (GQA); for MLA the two launches
+        part_bytes = float(np.mean([wl.partial_bytes(w, L) for L in lens_at])) + wl.combine_bytes(w)
         part_ms = float(np.mean(partial_ms))
         peak, tflops_peak, peak_kind = measured_peaks()
         achieved_gbs = part_bytes / (part_ms * 1e-3) / 1e9
-        kname = ("mla_partial_kernel" if w.kind == "mla" else
-                 "gqa_partial_nvfp4_kernel" if w.kv_dtype == "nvfp4" else
-                 f"gqa_partial_kernel<{w.d}>")
+        kname = ("mla_partial_kernel + combine_kernel" if w.kind == "mla" else
+                 "gqa_partial_nvfp4_kernel (fused combine)" if w.kv_dtype == "nvfp4" else
+                 f"gqa_partial_kernel<{w.d}> (fused combine)")
         flops = float(np.mean([wl.partial_flops(w, L) for L in lens_at]))
         achieved_tf = flops / (part_ms * 1e-3) / 1e12
         hbm = {"achieved": achieved_gbs, "peak": peak, "unit": "GB/s", "frac": achieved_gbs / peak}
@@ -446,9 +455,9 @@ def run_helix(args):
             "config": dict(config_of(w, lens), parallelism=f"replicas x{world}"),
             "achieved_hbm_tbs": step_bytes / (ms_step * 1e-3) / 1e12 * world,
             "step_bytes": step_bytes,
-            "kernels_us": {"partial": part_ms * 1e3,
-                           "append_combine_and_gaps": ms_step * 1e3 - part_ms * 1e3},
-            "gpu_launches": 3 * K,
+            "kernels_us": {"partial_and_combine": part_ms * 1e3,
+                           "append_and_gaps": ms_step * 1e3 - part_ms * 1e3},
+            "gpu_launches": (3 if w.kind == "mla" else 2) * K,
             "roofline": roof,
             "e2e": e2e,
             "clocks": clk,

@@ -182,6 +182,24 @@ helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads,
                                 int32_t o_dtype, float* lse_out, helix_stream_t stream);
 
 /*
+ * helix_attn_partial followed by helix_attn_combine, in ONE launch for GQA caches: the CTA that
+ * finishes the last of the kvp shards of a (request, KV head) group merges that group's rows into
+ * o_out / lse_out in the same kernel (the same arithmetic as helix_attn_combine, bit for bit).
+ * o_partial / lse still receive the per-shard results. For MLA caches the merge of a request
+ * (128 x 512 per shard) is too large for one CTA and this call issues the two launches.
+ *   arguments as helix_attn_partial + helix_attn_combine (o_dtype 0 bf16, 1 fp32; lse_out may be
+ *   NULL); the workspace is the one helix_attn_workspace_size reports.
+ * This is the step the paper summary describes for short contexts too (below about 4K tokens Helix
+ * degenerates to data-parallel attention): with kvp = 1 the merge is the identity and the step is
+ * one launch.
+ */
+helix_status helix_attn_partial_combine(const helix_kv_cache* cache, const void* q,
+                                        int32_t num_q_heads, float softmax_scale,
+                                        float* o_partial, float* lse, void* o_out,
+                                        int32_t o_dtype, float* lse_out, void* workspace,
+                                        size_t workspace_bytes, helix_stream_t stream);
+
+/*
  * helix_attn_partial restricted to the requests [b_begin, b_end) (0 <= b_begin <= b_end <= batch).
  * q, o_partial and lse keep their full shapes and indexing; rows of other requests are neither read
  * nor written. Same workspace as helix_attn_partial: calls sharing a workspace must be ordered on
@@ -219,6 +237,28 @@ helix_status helix_attn_overlapped(const helix_kv_cache* cache, const void* q, i
                                    void* workspace, size_t workspace_bytes,
                                    helix_stream_t stream_a, helix_stream_t stream_b,
                                    const helix_event_t* events);
+
+/*
+ * The HOP-B analogue for a whole decode step: as helix_attn_overlapped, and the append of each
+ * request group's new tokens also runs on stream_b, overlapping the previous group's partial
+ * attention (the pages' batch-wise overlap, extended to the append).
+ *   k_new ... n_new  as helix_kv_append (all requests' rows);
+ *   group_n_valid    device int32 [min(n_groups, B)][B]: row g gives every request's number of
+ *                    new rows for group g's append (n_new for requests of group g, 0 otherwise;
+ *                    groups are contiguous, ceil(B / n_groups) requests each);
+ *   events           2 * min(n_groups, B) + 1 caller-created CUDA events.
+ * Order: B: append(0); then per group g: A waits for append(g), runs partial(g); B runs
+ * append(g+1), waits for partial(g), runs combine(g); finally A waits for B. Requests whose row has
+ * 0 new tokens are not touched by that append (their lengths are not even rewritten).
+ */
+helix_status helix_decode_overlapped(const helix_kv_cache* cache, const void* q,
+                                    int32_t num_q_heads, float softmax_scale, int32_t n_groups,
+                                    const void* k_new, const void* v_new, const void* k_new_scale,
+                                    const void* v_new_scale, int32_t n_new,
+                                    const int32_t* group_n_valid, float* o_partial, float* lse,
+                                    void* o_out, int32_t o_dtype, float* lse_out, void* workspace,
+                                    size_t workspace_bytes, helix_stream_t stream_a,
+                                    helix_stream_t stream_b, const helix_event_t* events);
 
 /*
  * helix_attn_partial for callers that cannot allocate device memory. The paper has no counterpart;

@@ -66,6 +66,8 @@ def _load():
     lib.helix_attn_partial_noalloc.restype = I32
     lib.helix_attn_combine.argtypes = [I32, I32, I32, I32, P, P, P, I32, P, P]
     lib.helix_attn_combine.restype = I32
+    lib.helix_attn_partial_combine.argtypes = [cache_p, P, I32, F32, P, P, P, I32, P, P, SZ, P]
+    lib.helix_attn_partial_combine.restype = I32
     lib.helix_attn_partial_range.argtypes = [cache_p, P, I32, F32, I32, I32, P, P, P, SZ, P]
     lib.helix_attn_partial_range.restype = I32
     lib.helix_attn_combine_range.argtypes = [I32, I32, I32, I32, I32, I32, P, P, P, I32, P, P]
@@ -73,6 +75,9 @@ def _load():
     lib.helix_attn_overlapped.argtypes = [cache_p, P, I32, F32, I32, P, P, P, I32, P, P, SZ, P, P,
                                           ctypes.POINTER(P)]
     lib.helix_attn_overlapped.restype = I32
+    lib.helix_decode_overlapped.argtypes = [cache_p, P, I32, F32, I32, P, P, P, P, I32, P, P, P, P,
+                                            I32, P, P, SZ, P, P, ctypes.POINTER(P)]
+    lib.helix_decode_overlapped.restype = I32
     lib.helix_status_string.argtypes = [I32]
     lib.helix_status_string.restype = ctypes.c_char_p
     lib.helix_version.argtypes = []
@@ -242,6 +247,32 @@ def combine(o_partial: torch.Tensor, lse: torch.Tensor, out=None, lse_out=None,
     return out, lse_out
 
 
+def partial_combine(cache: KVCache, q: torch.Tensor, softmax_scale: float, o_partial=None,
+                    lse=None, out=None, lse_out=None, out_dtype=torch.bfloat16, workspace=None,
+                    stream=None):
+    """Partial attention and the LSE combine in one launch for GQA caches
+    (``helix_attn_partial_combine``). Returns (O, LSE)."""
+    B, Hq, _ = q.shape
+    dev = q.device
+    if o_partial is None:
+        o_partial = torch.empty(cache.kvp, B, Hq, cache.v_dim, dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty(cache.kvp, B, Hq, dtype=torch.float32, device=dev)
+    if out is None:
+        out = torch.empty(B, Hq, cache.v_dim, dtype=out_dtype, device=dev)
+    if lse_out is None:
+        lse_out = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = cache.workspace(Hq)
+    o_dtype = 0 if out.dtype == torch.bfloat16 else 1
+    _check(lib.helix_attn_partial_combine(ctypes.byref(cache.struct), _ptr(q), Hq,
+                                          float(softmax_scale), _ptr(o_partial), _ptr(lse),
+                                          _ptr(out), o_dtype, _ptr(lse_out), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream)), "helix_attn_partial_combine")
+    return out, lse_out
+
+
 def partial_range(cache: KVCache, q: torch.Tensor, softmax_scale: float, b_begin: int, b_end: int,
                   o_partial: torch.Tensor, lse: torch.Tensor, workspace=None, stream=None):
     """``helix_attn_partial_range``: partial attention of requests [b_begin, b_end) only, written
@@ -270,16 +301,32 @@ def combine_range(o_partial: torch.Tensor, lse: torch.Tensor, b_begin: int, b_en
 
 
 class Overlap:
-    """The second stream and the events ``helix_attn_overlapped`` needs, created once."""
+    """The second stream and the events ``helix_attn_overlapped`` / ``helix_decode_overlapped``
+    need, created once (2 * n_groups + 1 events: enough for either call)."""
 
     def __init__(self, n_groups: int, device=None):
         self.n_groups = int(n_groups)
+        self.device = device
         self.stream_b = torch.cuda.Stream(device=device)
         cur = torch.cuda.current_stream(device)
-        self.events = [torch.cuda.Event() for _ in range(self.n_groups + 1)]
+        self.events = [torch.cuda.Event() for _ in range(2 * self.n_groups + 1)]
         for e in self.events:  # torch creates the CUDA event lazily, on its first record
             e.record(cur)
         self._handles = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
+        self._nvalid = {}
+
+    def group_n_valid(self, batch: int, n_new: int, device):
+        """int32 [groups][batch]: n_new for the requests of group g in row g, 0 elsewhere."""
+        key = (batch, n_new)
+        if key not in self._nvalid:
+            g = min(self.n_groups, batch)
+            per = -(-batch // g)
+            t = torch.zeros(g, batch, dtype=torch.int32)
+            for i in range(g):
+                t[i, i * per:min(batch, (i + 1) * per)] = n_new
+            self._nvalid[key] = t.to(device)
+        return self._nvalid[key]
+
 
 
 def overlapped(cache: KVCache, q: torch.Tensor, softmax_scale: float, overlap: Overlap,
@@ -310,11 +357,44 @@ def overlapped(cache: KVCache, q: torch.Tensor, softmax_scale: float, overlap: O
     return out, lse_out
 
 
+def decode_overlapped(cache: KVCache, q: torch.Tensor, softmax_scale: float, overlap: Overlap,
+                      k_new, v_new=None, k_scale=None, v_scale=None, o_partial=None, lse=None,
+                      out=None, lse_out=None, out_dtype=torch.bfloat16, workspace=None,
+                      stream=None):
+    """HOP-B analogue of a whole decode step (``helix_decode_overlapped``): per request group the
+    append and the combine run on ``overlap.stream_b``, overlapping the neighbouring groups'
+    partial attention on ``stream``. Returns (O, LSE)."""
+    B, Hq, _ = q.shape
+    dev = q.device
+    n_new = int(k_new.shape[1])
+    if o_partial is None:
+        o_partial = torch.empty(cache.kvp, B, Hq, cache.v_dim, dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty(cache.kvp, B, Hq, dtype=torch.float32, device=dev)
+    if out is None:
+        out = torch.empty(B, Hq, cache.v_dim, dtype=out_dtype, device=dev)
+    if lse_out is None:
+        lse_out = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = cache.workspace(Hq)
+    gnv = overlap.group_n_valid(B, n_new, dev)
+    o_dtype = 0 if out.dtype == torch.bfloat16 else 1
+    _check(lib.helix_decode_overlapped(ctypes.byref(cache.struct), _ptr(q), Hq,
+                                       float(softmax_scale), overlap.n_groups, _ptr(k_new),
+                                       _ptr(v_new), _ptr(k_scale), _ptr(v_scale), n_new, _ptr(gnv),
+                                       _ptr(o_partial), _ptr(lse), _ptr(out), o_dtype,
+                                       _ptr(lse_out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream), _stream(overlap.stream_b),
+                                       overlap._handles), "helix_decode_overlapped")
+    return out, lse_out
+
+
 def decode_step(cache: KVCache, q, k_new, v_new=None, softmax_scale=None, k_scale=None,
                 v_scale=None, o_partial=None, lse=None, out=None, lse_out=None, stream=None):
-    """One decode-attention layer step: append the new token, partial attention, combine."""
+    """One decode-attention layer step: append the new token, then partial attention and the
+    combine (one launch for GQA caches, ``helix_attn_partial_combine``). Returns (O, LSE)."""
     if softmax_scale is None:
         softmax_scale = cache.head_dim ** -0.5
     append(cache, k_new, v_new, k_scale, v_scale, stream=stream)
-    o_partial, lse = partial(cache, q, softmax_scale, o_partial, lse, stream=stream)
-    return combine(o_partial, lse, out, lse_out, stream=stream)
+    return partial_combine(cache, q, softmax_scale, o_partial, lse, out, lse_out, stream=stream)

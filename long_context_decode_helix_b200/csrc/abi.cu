@@ -108,11 +108,14 @@ helix_status check_cache(const helix_kv_cache* c) {
   return HELIX_OK;
 }
 
+// Workspace layout: [unit tickets][group tickets (GQA fused combine)][segment records]
 struct PartialPlan {
   int grid;
   int units;
   size_t ticket_bytes;
+  size_t gticket_bytes;
   size_t seg_bytes;
+  size_t total() const { return ticket_bytes + gticket_bytes + seg_bytes; }
 };
 
 helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan* plan) {
@@ -130,6 +133,7 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
     plan->grid = (sms / 2) * 2;  // clusters of two CTAs
     if (plan->grid < 2) return HELIX_ERR_UNSUPPORTED;
     plan->ticket_bytes = (((size_t)plan->units * 2 * sizeof(int32_t)) + 255) & ~size_t(255);
+    plan->gticket_bytes = 0;
     plan->seg_bytes = (size_t)(plan->grid / 2) * 2 * 2 * mla_segment_record_floats() * sizeof(float);
     return HELIX_OK;
   }
@@ -146,6 +150,8 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
   if (smem > (size_t)max_smem) return HELIX_ERR_CAPACITY;
   plan->grid = sms;
   plan->ticket_bytes = (((size_t)plan->units * sizeof(int32_t)) + 255) & ~size_t(255);
+  plan->gticket_bytes =
+      (((size_t)c->batch * c->num_kv_heads * sizeof(int32_t)) + 255) & ~size_t(255);
   const size_t rec = nvfp4 ? gqa_nvfp4_segment_record_floats()
                            : gqa_segment_record_floats(c->head_dim);
   plan->seg_bytes = (size_t)plan->grid * 2 * rec * sizeof(float);
@@ -263,14 +269,21 @@ helix_status helix_attn_workspace_size(const helix_kv_cache* c, int32_t num_q_he
   PartialPlan plan;
   helix_status st = plan_partial(c, num_q_heads, &plan);
   if (st != HELIX_OK) return st;
-  *bytes = plan.ticket_bytes + plan.seg_bytes;
+  *bytes = plan.total();
   return HELIX_OK;
 }
 
-helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
-                                      int32_t num_q_heads, float softmax_scale, int32_t b_begin,
-                                      int32_t b_end, float* o_partial, float* lse, void* workspace,
-                                      size_t workspace_bytes, helix_stream_t stream) {
+}  // extern "C"
+
+namespace helix {
+namespace {
+
+// The partial attention of requests [b_begin, b_end); with o_out non-null (GQA only) the kernel
+// also merges the shards of every KV-head group into o_out / lse_out (fused combine).
+helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                          float softmax_scale, int32_t b_begin, int32_t b_end, float* o_partial,
+                          float* lse, void* workspace, size_t workspace_bytes, void* o_out,
+                          int32_t o_dtype, float* lse_out, cudaStream_t stream) {
   if (c == nullptr || b_begin < 0 || b_end < b_begin || b_end > c->batch)
     return HELIX_ERR_INVALID_ARG;
   PartialPlan plan;
@@ -280,7 +293,10 @@ helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
     return HELIX_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o_partial) || !aligned4(lse) || !aligned16(workspace))
     return HELIX_ERR_INVALID_ARG;
-  if (workspace_bytes < plan.ticket_bytes + plan.seg_bytes) return HELIX_ERR_INVALID_ARG;
+  if (workspace_bytes < plan.total()) return HELIX_ERR_INVALID_ARG;
+  if (o_out != nullptr && (c->kind != HELIX_ATTN_GQA || (o_dtype != 0 && o_dtype != 1) ||
+                           !aligned16(o_out) || !aligned4(lse_out)))
+    return HELIX_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return HELIX_ERR_INVALID_ARG;
   if (b_end == b_begin) return HELIX_OK;
   // units are ordered request-major, so a request range is a contiguous unit range
@@ -295,7 +311,8 @@ helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
     m.o_part = o_partial;
     m.lse = lse;
     m.tickets = reinterpret_cast<int32_t*>(workspace);
-    m.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes);
+    m.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes +
+                                     plan.gticket_bytes);
     m.err = c->err_word;
     m.B = c->batch;
     m.kvp = c->kvp;
@@ -304,15 +321,15 @@ helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
     m.units = units;
     m.u0 = u0;
     m.scale_log2 = softmax_scale * 1.4426950408889634f;
-    // latent pool as [pages * 64 rows][576], boxes of 64 columns x 32 rows; q as [B * 128][576],
+    // latent pool as [pages * 64 rows][576], boxes of 64 columns x 64 rows; q as [B * 128][576],
     // boxes of 64 columns x 128 rows; 128-byte swizzle for the tensor-core operand layout
     CUtensorMap tmC, tmQ;
     if (!encode_rows_map(&tmC, c->k_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
-                         (uint64_t)c->num_pages * 64, 64, 32) ||
+                         (uint64_t)c->num_pages * 64, 64, 64) ||
         !encode_rows_map(&tmQ, const_cast<void*>(q), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
                          (uint64_t)c->batch * 128, 64, 128))
       return HELIX_ERR_CUDA;
-    return mla_partial_launch(tmC, tmQ, m, plan.grid, reinterpret_cast<cudaStream_t>(stream));
+    return mla_partial_launch(tmC, tmQ, m, plan.grid, stream);
   }
 
   GqaParams p{};
@@ -322,7 +339,13 @@ helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
   p.o_part = o_partial;
   p.lse = lse;
   p.tickets = reinterpret_cast<int32_t*>(workspace);
-  p.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes);
+  p.gtickets =
+      reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes);
+  p.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes +
+                                   plan.gticket_bytes);
+  p.o_out = o_out;
+  p.o_dtype = o_dtype;
+  p.lse_out = o_out != nullptr ? lse_out : nullptr;
   p.err = c->err_word;
   p.B = c->batch;
   p.Hq = num_q_heads;
@@ -340,7 +363,7 @@ helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
     p.k_scale = reinterpret_cast<const uint8_t*>(c->k_scale);
     p.v_codes = reinterpret_cast<const uint8_t*>(c->v_pool);
     p.v_scale = reinterpret_cast<const uint8_t*>(c->v_scale);
-    return gqa_partial_nvfp4_launch(p, plan.grid, reinterpret_cast<cudaStream_t>(stream));
+    return gqa_partial_nvfp4_launch(p, plan.grid, stream);
   }
 
   const uint64_t rows = (uint64_t)c->num_pages * c->num_kv_heads * c->page_tokens;
@@ -350,7 +373,43 @@ helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
       !encode_rows_map(&tmV, c->v_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c->head_dim, rows,
                        64, 64))
     return HELIX_ERR_CUDA;
-  return gqa_partial_bf16_launch(tmK, tmV, p, plan.grid, reinterpret_cast<cudaStream_t>(stream));
+  return gqa_partial_bf16_launch(tmK, tmV, p, plan.grid, stream);
+}
+
+}  // namespace
+}  // namespace helix
+
+extern "C" {
+
+helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
+                                      int32_t num_q_heads, float softmax_scale, int32_t b_begin,
+                                      int32_t b_end, float* o_partial, float* lse, void* workspace,
+                                      size_t workspace_bytes, helix_stream_t stream) {
+  return partial_impl(c, q, num_q_heads, softmax_scale, b_begin, b_end, o_partial, lse, workspace,
+                      workspace_bytes, nullptr, 0, nullptr,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+helix_status helix_attn_partial_combine(const helix_kv_cache* c, const void* q,
+                                        int32_t num_q_heads, float softmax_scale,
+                                        float* o_partial, float* lse, void* o_out,
+                                        int32_t o_dtype, float* lse_out, void* workspace,
+                                        size_t workspace_bytes, helix_stream_t stream) {
+  if (c == nullptr) return HELIX_ERR_INVALID_ARG;
+  if (c->kind == HELIX_ATTN_GQA)
+    return partial_impl(c, q, num_q_heads, softmax_scale, 0, c->batch, o_partial, lse, workspace,
+                        workspace_bytes, o_out, o_dtype, lse_out,
+                        reinterpret_cast<cudaStream_t>(stream));
+  // MLA: a whole request's 128 x 512 merge is too large for one CTA; two launches
+  if (o_out == nullptr || (o_dtype != 0 && o_dtype != 1) || !aligned16(o_out) ||
+      !aligned4(lse_out))
+    return HELIX_ERR_INVALID_ARG;
+  helix_status st = partial_impl(c, q, num_q_heads, softmax_scale, 0, c->batch, o_partial, lse,
+                                 workspace, workspace_bytes, nullptr, 0, nullptr,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (st != HELIX_OK) return st;
+  return helix_attn_combine(c->kvp, c->batch, num_q_heads, c->v_dim, o_partial, lse, o_out,
+                            o_dtype, lse_out, stream);
 }
 
 helix_status helix_attn_partial(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
@@ -423,6 +482,66 @@ helix_status helix_attn_overlapped(const helix_kv_cache* c, const void* q, int32
   }
   // join: stream A waits for the last combine, so the caller needs to order only against A
   auto done = reinterpret_cast<cudaEvent_t>(events[n_groups]);
+  if (cudaEventRecord(done, sb) != cudaSuccess || cudaStreamWaitEvent(sa, done, 0) != cudaSuccess)
+    return HELIX_ERR_CUDA;
+  return HELIX_OK;
+}
+
+helix_status helix_decode_overlapped(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                                    float softmax_scale, int32_t n_groups, const void* k_new,
+                                    const void* v_new, const void* k_new_scale,
+                                    const void* v_new_scale, int32_t n_new,
+                                    const int32_t* group_n_valid, float* o_partial, float* lse,
+                                    void* o_out, int32_t o_dtype, float* lse_out, void* workspace,
+                                    size_t workspace_bytes, helix_stream_t stream_a,
+                                    helix_stream_t stream_b, const helix_event_t* events) {
+  if (c == nullptr || events == nullptr || n_groups < 1 || group_n_valid == nullptr)
+    return HELIX_ERR_INVALID_ARG;
+  if (stream_a == stream_b || n_new < 1) return HELIX_ERR_INVALID_ARG;
+  const int B = c->batch;
+  const int groups = n_groups < B ? n_groups : B;
+  for (int e = 0; e < 2 * groups + 1; ++e)
+    if (events[e] == nullptr) return HELIX_ERR_INVALID_ARG;
+  PartialPlan plan;
+  helix_status st = plan_partial(c, num_q_heads, &plan);
+  if (st != HELIX_OK) return st;
+  if (q == nullptr || o_partial == nullptr || lse == nullptr || workspace == nullptr ||
+      o_out == nullptr || (o_dtype != 0 && o_dtype != 1) || c->v_dim % 4 != 0 ||
+      !aligned16(o_out) || !aligned4(lse_out) || !aligned4(group_n_valid))
+    return HELIX_ERR_INVALID_ARG;
+  const int per = (B + groups - 1) / groups;
+  const int ng = (B + per - 1) / per;  // groups actually formed
+  auto sa = reinterpret_cast<cudaStream_t>(stream_a);
+  auto sb = reinterpret_cast<cudaStream_t>(stream_b);
+  auto ev_app = [&](int g) { return reinterpret_cast<cudaEvent_t>(events[g]); };
+  auto ev_part = [&](int g) { return reinterpret_cast<cudaEvent_t>(events[groups + g]); };
+  auto append_group = [&](int g) -> helix_status {  // on stream B; row g of group_n_valid
+    helix_status s2 = helix_kv_append(c, k_new, v_new, k_new_scale, v_new_scale, n_new,
+                                      group_n_valid + (size_t)g * B, stream_b);
+    if (s2 != HELIX_OK) return s2;
+    return cudaEventRecord(ev_app(g), sb) == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
+  };
+  st = append_group(0);
+  if (st != HELIX_OK) return st;
+  for (int g = 0; g < ng; ++g) {
+    const int b0 = g * per, b1 = b0 + per < B ? b0 + per : B;
+    // stream A: group g's partial once its new tokens are in the cache
+    if (cudaStreamWaitEvent(sa, ev_app(g), 0) != cudaSuccess) return HELIX_ERR_CUDA;
+    st = helix_attn_partial_range(c, q, num_q_heads, softmax_scale, b0, b1, o_partial, lse,
+                                  workspace, workspace_bytes, stream_a);
+    if (st != HELIX_OK) return st;
+    if (cudaEventRecord(ev_part(g), sa) != cudaSuccess) return HELIX_ERR_CUDA;
+    // stream B: the next group's append overlaps this partial, then this group's combine
+    if (g + 1 < ng) {
+      st = append_group(g + 1);
+      if (st != HELIX_OK) return st;
+    }
+    if (cudaStreamWaitEvent(sb, ev_part(g), 0) != cudaSuccess) return HELIX_ERR_CUDA;
+    st = helix_attn_combine_range(c->kvp, B, num_q_heads, c->v_dim, b0, b1, o_partial, lse, o_out,
+                                  o_dtype, lse_out, stream_b);
+    if (st != HELIX_OK) return st;
+  }
+  auto done = reinterpret_cast<cudaEvent_t>(events[2 * groups]);
   if (cudaEventRecord(done, sb) != cudaSuccess || cudaStreamWaitEvent(sa, done, 0) != cudaSuccess)
     return HELIX_ERR_CUDA;
   return HELIX_OK;

@@ -131,8 +131,10 @@ __device__ __forceinline__ int rows_of(const AppendParams& p, int b) {
 }
 
 __device__ void update_lengths(const AppendParams& p, int b) {
+  const int rows = rows_of(p, b);
+  if (rows == 0) return;  // leave the lengths of requests without new rows untouched
   const long long S_old = p.seq_lens[b];
-  const long long S_new = S_old + rows_of(p, b);
+  const long long S_new = S_old + rows;
   for (int s = 0; s < p.kvp; ++s) {
     const long long add = count_on_shard(S_new, s, p) - count_on_shard(S_old, s, p);
     p.shard_lens[s * p.B + b] += (int)add;

@@ -30,6 +30,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "combine_row.cuh"
 #include "device_common.cuh"
 #include "internal.h"
 
@@ -63,6 +64,7 @@ struct SmemTail {
   float lstat[kConsumerWarps][kRows];
   float lbstat[kConsumerWarps][kRows];
   int flag;
+  int gflag;
   int abort_;
 };
 
@@ -162,6 +164,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t row0 = ((size_t)s * p.B + b) * p.Hq + (size_t)k * p.G;
     for (int i = tid; i < p.G * D; i += kThreads) p.o_part[row0 * D + i] = 0.f;
     for (int i = tid; i < p.G; i += kThreads) p.lse[row0 + i] = -INFINITY;
+    if (p.o_out != nullptr)
+      fused_group_combine(p, bk, &tail->gflag, [] { __syncthreads(); }, tid, warp, lane,
+                          kThreads / 32);
   }
   const int Geff = (int)min((long long)gridDim.x, W);
   if ((int)blockIdx.x >= Geff) return;
@@ -515,6 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       const size_t orow = ((size_t)s_u * p.B + b_u) * p.Hq + (size_t)k_u * p.G + r;
       const bool whole = seg_begin == pre[u] && g + 1 == pre[u + 1];
+      bool unit_written = whole;  // this CTA wrote the unit's final O_partial / lse
       if (whole) {
         if (r < p.G) {
           const float inv = LB > 0.f ? 1.f / LB : 0.f;
@@ -549,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tail->flag = (ticket == c_hi - c_lo) ? 1 : 0;
         }
         named_barrier_sync(1, kConsumerWarps * 32);
+        unit_written = tail->flag != 0;
         if (tail->flag) {  // last arriver merges every segment of this unit
           __threadfence();
           float Mm = -INFINITY;
@@ -589,6 +596,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tid == 0) p.tickets[u] = 0;  // ready for the next launch
         }
       }
+      if (p.o_out != nullptr && unit_written)
+        fused_group_combine(p, (int)((u + p.u0) / p.kvp), &tail->gflag,
+                            [] { named_barrier_sync(1, kConsumerWarps * 32); }, tid, warp, lane,
+                            kConsumerWarps);
       named_barrier_sync(1, kConsumerWarps * 32);
       reset_state();
       seg_begin = g + 1;

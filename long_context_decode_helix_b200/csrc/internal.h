@@ -28,6 +28,12 @@ struct GqaParams {
   int B, Hq, Hkv, G, D, kvp, max_pages, num_pages, units;
   int u0;                     // first unit of this launch (a request boundary)
   float scale_log2;  // softmax_scale * log2(e)
+  // fused combine (o_out non-null): the CTA that finishes the last of the kvp units of a group
+  // (b, k) merges the group's rows into o_out / lse_out
+  void* o_out;                // [B][Hq][D], bf16 (o_dtype 0) or fp32 (1)
+  float* lse_out;             // [B][Hq], may be null
+  int32_t* gtickets;          // [B * Hkv], zero between launches
+  int o_dtype;
 };
 
 size_t gqa_partial_smem_bytes(int head_dim, int units);  // bf16 kernel

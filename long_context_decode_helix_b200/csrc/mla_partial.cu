@@ -11,16 +11,18 @@
 //
 // Sizes force a two-CTA design. O for 128 heads x 512 columns in fp32 fills all 512 TMEM columns
 // and q (128 x 576 bf16) alone is 144 KiB, so one CTA cannot hold q, a score tile and O. A cluster
-// of two CTAs works on the same 32-token tiles:
+// of two CTAs works on the same 64-token tiles (one page each):
 //   * CTA r keeps half of q's contraction (head-dim elements [288 r, 288 r + 288)) in shared memory
-//     and computes a partial score tile S_r = q[:, half] C[:, half]^T (M = 128 heads, N = 32 tokens,
-//     K = 288) into TMEM;
+//     and computes a partial score tile S_r = q[:, half] C[:, half]^T (M = 128 heads, N = 64 tokens,
+//     K = 288) into TMEM. A tcgen05.mma of M = 128 costs about the same for any N up to 128
+//     (measured: about 110 SM cycles for one K = 16 step), so the score tile is as wide as the
+//     shared-memory budget allows;
 //   * the two CTAs swap their partials through distributed shared memory: st.async stores into the
 //     peer's exchange buffer complete a transaction count on the peer's mbarrier, and the buffer is
 //     handed back with a relaxed remote arrive (no multicast loads anywhere), so both hold the same
-//     full S;
+//     full S. One exchange buffer serves the tiles in turn;
 //   * each CTA runs the same online softmax, writes P (bf16) back into TMEM and accumulates O for
-//     its half of the value columns (M = 128, N = 256, K = 32 tokens) in 256 TMEM columns with the
+//     its half of the value columns (M = 128, N = 256, K = 64 tokens) in 256 TMEM columns with the
 //     TS form of the MMA (A = P from TMEM, B = V read straight from the latent tile it already holds,
 //     MN-major).
 // Each CTA loads five 64-column chunks of every latent row (chunks 0-4 or 4-8), so together the pair
@@ -29,13 +31,13 @@
 // Warps: 0-7 softmax / epilogue in two groups of four (group g takes the tiles i with i % 2 == g,
 // so two tiles are in the softmax at once; thread h of a group owns head h = TMEM lane h), 8 TMA
 // producer, 9 MMA issuer (one elected thread, which issues whichever of the next S tile or the next
-// P V product is ready) and TMEM allocator. Score tiles have four TMEM buffers, so the tensor core
-// runs ahead of the softmax. The groups share one reference maximum per head, handed from the owner
+// P V product is ready) and TMEM allocator. Each group has its own TMEM score buffer, so the tensor
+// core computes the next tile's scores while a group works on its tile. The groups share one reference maximum per head, handed from the owner
 // of tile i-1 to the owner of tile i through shared memory and a named barrier; each group keeps its
 // own running sum, and the two are merged at the end of a segment. O is rescaled lazily: the exponent base only moves when
 // a row maximum grows by more than 8 (in base-2 units), so weights stay below 2^8 and the 256-column
 // TMEM rescale is rare. Work is split over the (request, shard) units exactly as in the GQA kernel:
-// each cluster takes an equal contiguous range of 32-token tiles; split units are merged by the last
+// each cluster takes an equal contiguous range of 64-token tiles; split units are merged by the last
 // arriving cluster, per value half.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -51,18 +53,18 @@ namespace {
 
 constexpr int kHeads = 128;
 constexpr int kDV = 512, kHalfDV = 256;  // V: the first 512 of the 576 latent columns
-constexpr int kTok = 32;                   // tokens per tile
+constexpr int kTok = 64;                   // tokens per tile (one page)
 constexpr int kPageTok = 64;               // tokens per page
 constexpr int kChunks = 5;                 // 64-column chunks of a latent row per CTA
 constexpr int kKSteps = 18;                // 288 / 16
-constexpr int kNS = 5;                     // tile stages
-constexpr int kNX = 2;                     // score-exchange buffers
-constexpr int kStageBytes = kTok * kChunks * 128;     // 20 KiB
+constexpr int kNS = 2;                     // tile stages
+constexpr int kNX = 1;                     // score-exchange buffers (the groups take turns)
+constexpr int kStageBytes = kTok * kChunks * 128;     // 40 KiB
 constexpr int kQBytes = kHeads * kChunks * 128;        // 80 KiB
-constexpr int kSBuf = 4;                               // score-tile buffers in TMEM
-constexpr uint32_t kSCol = 256, kPCol = 384;           // TMEM columns: O [0,256), S 4x32, P 2x16
+constexpr int kSBuf = 2;                               // score-tile buffers in TMEM
+constexpr uint32_t kSCol = 256, kPCol = 384;           // TMEM columns: O [0,256), S 2x64, P 2x32
 constexpr int kXStride = kTok + 4;                     // padded fp32 row of the exchange buffer
-constexpr int kXBytes = kHeads * kXStride * 4;         // 18 KiB
+constexpr int kXBytes = kHeads * kXStride * 4;         // 34 KiB
 // warps 0-7: two softmax groups of four (group g takes the tiles i with i % 2 == g)
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 10 * 32;
@@ -175,16 +177,6 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
       : "memory");
 }
-// 16 consecutive 32-bit columns of this thread's TMEM lane
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, bool accumulate) {
   asm volatile(
@@ -208,6 +200,43 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 64 consecutive fp32 columns of this thread's TMEM lane (two 32-column loads, one wait)
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+#pragma unroll
+  for (int half = 0; half < 2; ++half)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[32 * half + 0]), "=r"(r[32 * half + 1]), "=r"(r[32 * half + 2]),
+          "=r"(r[32 * half + 3]), "=r"(r[32 * half + 4]), "=r"(r[32 * half + 5]),
+          "=r"(r[32 * half + 6]), "=r"(r[32 * half + 7]), "=r"(r[32 * half + 8]),
+          "=r"(r[32 * half + 9]), "=r"(r[32 * half + 10]), "=r"(r[32 * half + 11]),
+          "=r"(r[32 * half + 12]), "=r"(r[32 * half + 13]), "=r"(r[32 * half + 14]),
+          "=r"(r[32 * half + 15]), "=r"(r[32 * half + 16]), "=r"(r[32 * half + 17]),
+          "=r"(r[32 * half + 18]), "=r"(r[32 * half + 19]), "=r"(r[32 * half + 20]),
+          "=r"(r[32 * half + 21]), "=r"(r[32 * half + 22]), "=r"(r[32 * half + 23]),
+          "=r"(r[32 * half + 24]), "=r"(r[32 * half + 25]), "=r"(r[32 * half + 26]),
+          "=r"(r[32 * half + 27]), "=r"(r[32 * half + 28]), "=r"(r[32 * half + 29]),
+          "=r"(r[32 * half + 30]), "=r"(r[32 * half + 31])
+        : "r"(taddr + 32 * half));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 32 consecutive 32-bit columns of this thread's TMEM lane (raw bits)
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+      "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
+      "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
+      "r"(v[30]), "r"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
@@ -257,7 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* q_s = smem;                                   // [5 chunks][128 rows][128 B]
-  uint8_t* stage_s = q_s + kQBytes;                      // [kNS][5 chunks][32 rows][128 B]
+  uint8_t* stage_s = q_s + kQBytes;                      // [kNS][5 chunks][64 rows][128 B]
   float* x_s = reinterpret_cast<float*>(stage_s + kNS * kStageBytes);  // [kNX][128][kXStride]
   MlaTail* tail = reinterpret_cast<MlaTail*>(x_s + kNX * kHeads * kXStride);
   int* pre = reinterpret_cast<int*>(tail + 1);
@@ -306,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tail->flag = 0;
     tail->abort_ = 0;
     fence_mbar_init();
-    // arm the exchange barriers for the first kNX tiles (128 rows x 32 fp32 scores each)
+    // arm the exchange barrier for the first tile (128 rows x 64 fp32 scores)
     for (int i = 0; i < kNX; ++i) mbar_arrive_expect_tx(&tail->x_full[i], kHeads * kTok * 4);
   }
   if (warp == kMmaWarp) {  // allocate all 512 TMEM columns (one CTA per SM)
@@ -397,7 +426,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         const int lt = (int)(g - pre[u]);  // tile within the unit
-        const int page = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + lt / 2);
+        const int page = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + lt);
         if (page < 0 || page >= p.num_pages) {
           raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
           tail->stage_ok[stage] = 0;
@@ -406,7 +435,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tail->stage_ok[stage] = 1;
           mbar_arrive_expect_tx(&tail->stage_full[stage], kStageBytes);
           uint8_t* st = stage_s + stage * kStageBytes;
-          const int row = page * kPageTok + (lt & 1) * kTok;
+          const int row = page * kPageTok;
           for (int c = 0; c < kChunks; ++c)
             tma_load_2d(st + c * kTok * 128, &tmC, (4 * rank + c) * 64, row,
                         &tail->stage_full[stage]);
@@ -447,7 +476,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               // 32-row chunk (4 KiB) apart, 8-token groups 1 KiB apart
               const uint64_t bdesc =
                   smem_desc(vbase + ks * 16 * 128, kTok * 128, 1024, kSwizzle128);
-              tc_mma_ts(tmem, tmem + kPCol + pb * 16 + ks * 8, bdesc, idPV, !(fresh && ks == 0));
+              tc_mma_ts(tmem, tmem + kPCol + pb * (kTok / 2) + ks * 8, bdesc, idPV,
+                        !(fresh && ks == 0));
             }
             tc_commit(&tail->stage_empty[st]);
             tc_commit(&tail->p_empty[pb]);
@@ -555,7 +585,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       m_own = -INFINITY;
       l_own = 0.f;
     };
-    float sv[32];
+    float sv[kTok];
     for (long long i = grp; i < n_tiles; i += 2) {
       const long long g = g_begin + i;
       unit_of(g);
@@ -574,7 +604,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool tile_ok = tail->stage_ok[st_i] != 0;
       if (!dead) {
         tc_fence_after();
-        tmem_ld32(tl + kSCol + sb * kTok, sv);
+        tmem_ld64(tl + kSCol + sb * kTok, sv);
         tc_fence_before();
       } else {
 #pragma unroll
@@ -582,20 +612,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->s_empty[sb]);
-      if (i >= 2) wwait(&tail->x_free[grp], (uint32_t)(((i - 2) >> 1) & 1), true);
+      // the one exchange buffer serves the tiles in turn: tile i-1's scores must have been read
+      if (i >= 1) wwait(&tail->x_free[0], (uint32_t)((i - 1) & 1), true);
       {
-        const uint32_t dst = x_peer + (uint32_t)((grp * kHeads + h) * kXStride * 4);
+        const uint32_t dst = x_peer + (uint32_t)(h * kXStride * 4);
 #pragma unroll
         for (int c = 0; c < kTok; c += 4)
-          st_async_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3], xfull_peer + grp * 8);
+          st_async_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3], xfull_peer);
       }
       // the previous tile closed a segment owned by the other group: join its flush before this
       // tile's P can reach the MMA (its P V would overwrite O)
       if (fresh && i > 0) join_segment_end();
       // ---- B: add the peer's partial, softmax, P into TMEM ----
-      wwait(&tail->x_full[grp], (uint32_t)((i >> 1) & 1), true);
+      wwait(&tail->x_full[0], (uint32_t)(i & 1), true);
       {
-        const float* mine = x_s + (size_t)(grp * kHeads + h) * kXStride;
+        const float* mine = x_s + (size_t)h * kXStride;
 #pragma unroll
         for (int c = 0; c < kTok; c += 4) {
           const float4 v = *reinterpret_cast<const float4*>(mine + c);
@@ -605,12 +636,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           sv[c + 3] += v.w;
         }
       }
-      // re-arm this group's exchange barrier for tile i+2 (every thread here has observed tile
-      // i's phase), then hand the buffer back to the peer once its loads have returned
-      if (h == 0 && i + 2 < n_tiles) mbar_arrive_expect_tx(&tail->x_full[grp], kHeads * kTok * 4);
+      // re-arm the exchange barrier for tile i+1 (every thread of this group has observed tile i's
+      // phase; the peer sends tile i+1 only after this group's hand-back below), then hand the
+      // buffer back to the peer once its loads have returned
+      if (h == 0 && i + 1 < n_tiles) mbar_arrive_expect_tx(&tail->x_full[0], kHeads * kTok * 4);
       keep_alive(sv);
       __syncwarp();
-      if (lane == 0) remote_arrive_relaxed(xfree_peer + grp * 8);
+      if (lane == 0) remote_arrive_relaxed(xfree_peer);
       if (nvalid == kTok && tile_ok) {
 #pragma unroll
         for (int c = 0; c < kTok; ++c) sv[c] *= sl2;
@@ -622,7 +654,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       {  // tree reduction of the row maximum
         float t[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) t[c] = fmaxf(sv[c], sv[c + 16]);
+        for (int c = 0; c < 16; ++c) t[c] = fmaxf(fmaxf(sv[c], sv[c + 16]), fmaxf(sv[c + 32], sv[c + 48]));
 #pragma unroll
         for (int c = 0; c < 8; ++c) t[c] = fmaxf(t[c], t[c + 8]);
 #pragma unroll
@@ -658,13 +690,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         l_own = l_own > 0.f ? l_own * fast_exp2(m_own - mb) : 0.f;
         m_own = m_new;
       }
-      uint32_t pk[16];
+      uint32_t pk[kTok / 2];
       float ps[16];
 #pragma unroll
-      for (int c = 0; c < kTok; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         const float p0 = fast_exp2(sv[c] - mb), p1 = fast_exp2(sv[c + 1] - mb);
-        ps[c / 2] = p0 + p1;
+        const float p2 = fast_exp2(sv[c + 32] - mb), p3 = fast_exp2(sv[c + 33] - mb);
+        ps[c / 2] = (p0 + p1) + (p2 + p3);
         pk[c / 2] = pack_bf16x2(p0, p1);
+        pk[16 + c / 2] = pack_bf16x2(p2, p3);
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) ps[c] += ps[c + 8];
@@ -689,8 +723,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
       }
-      // P row h (32 bf16) into this thread's TMEM lane: the A operand of the P V product
-      if (!dead) tmem_st16(tl + kPCol + grp * 16, pk);
+      // P row h (64 bf16) into this thread's TMEM lane: the A operand of the P V product
+      if (!dead) tmem_st32u(tl + kPCol + grp * (kTok / 2), pk);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->p_full[grp]);

@@ -38,7 +38,7 @@ def _check(w, q, lens, res, label, heads=None):
 
 
 CASES = {
-    # several 32-token tiles and a partial tile per shard
+    # several 64-token tiles and a partial tile per shard
     "small": (MLA.with_(B=1, S=700, kvp=2), [700]),
     # one token, a partial page, empty shards (8 shards, 1 token)
     "ragged_empty": (MLA.with_(B=3, S=1000, kvp=8), [1000, 1, 77]),

@@ -122,3 +122,33 @@ def test_overlapped_orders_against_later_work_on_stream_a():
     assert np.isfinite(snap.cpu().numpy()).all()
     _check_requests(w, cache, q, lens, snap.cpu().numpy(), ser_lse.cpu().numpy(), range(w.B),
                     "after overlapped")
+
+
+@pytest.mark.parametrize("w,lens,groups", [(GQA, GQA_LENS, 2), (GQA, GQA_LENS, 5), (MLA, MLA_LENS, 2)],
+                         ids=["gqa-g2", "gqa-g5", "mla-g2"])
+def test_decode_overlapped_equals_the_serial_step(w, lens, groups):
+    """HOP-B with the append overlapped too: per request group the new token is appended on the
+    second stream while the previous group's partial runs. Same cache contents, lengths and (up to
+    the split rounding) outputs as the serial decode step."""
+    hx = _gpu.hx()
+    ca, q = _setup(w, [L - 1 for L in lens])
+    cb, _ = _setup(w, [L - 1 for L in lens])
+    rows = _gpu.new_rows(w, 0, w.S)
+    last = {k: torch.stack([v[b, lens[b] - 1] for b in range(w.B)])[:, None].contiguous()
+            for k, v in rows.items()}
+    out_a, lse_a = hx.decode_step(ca, q, last["k_new"], last.get("v_new"), w.softmax_scale,
+                                  out=torch.empty(w.B, w.Hq, w.dv, device="cuda"))
+    ov = hx.Overlap(groups)
+    out_b, lse_b = hx.decode_overlapped(cb, q, w.softmax_scale, ov, last["k_new"], last.get("v_new"),
+                                        out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ca["seq_lens"].tolist() == lens and cb["seq_lens"].tolist() == lens
+    assert torch.equal(ca["shard_lens"], cb["shard_lens"])
+    assert torch.equal(ca["k_pool"], cb["k_pool"])
+    if w.kind != "mla":
+        assert torch.equal(ca["v_pool"], cb["v_pool"])
+    assert (out_a - out_b).abs().max().item() < SPLIT_TOL_O
+    assert (lse_a - lse_b).abs().max().item() < SPLIT_TOL_LSE
+    _check_requests(w, cb, q, lens, out_b.cpu().numpy(), lse_b.cpu().numpy(), range(w.B),
+                    f"decode overlapped g={groups}")
+    assert ca.err_bits() == 0 and cb.err_bits() == 0

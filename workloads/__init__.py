@@ -68,6 +68,9 @@ class Workload:
     S_min: int | None = None  # lengths drawn uniformly in [S_min, S] when set
     rr_block: int = 16
     page_tokens: int = 64
+    # the final length the contiguous layout is sized for (C = ceil(S_final / P)); None = S. A
+    # decode loop that appends past S needs it, or the new tokens would fall off the last shard.
+    S_final: int | None = None
 
     @property
     def G(self) -> int:
@@ -79,7 +82,7 @@ class Workload:
 
     @property
     def contig_chunk(self) -> int:
-        return -(-self.S // self.kvp)
+        return -(-(self.S if self.S_final is None else self.S_final) // self.kvp)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
