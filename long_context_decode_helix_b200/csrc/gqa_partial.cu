@@ -44,6 +44,7 @@ constexpr int kGroups = 2;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kChunkBytes = kPage * 64 * 2;  // one 64-column half of a bf16 page-head: 8 KiB
 constexpr int kMergeSlots = 2;               // 16 x D fp32 buffers for the cross-warp merge
+constexpr int kMinPagesPerCta = 4;
 
 template <int D>
 struct GqaCfg {
@@ -168,7 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       fused_group_combine(p, bk, &tail->gflag, [] { __syncthreads(); }, tid, warp, lane,
                           kThreads / 32);
   }
-  const int Geff = (int)min((long long)gridDim.x, W);
+  // at least kMinPagesPerCta pages per CTA: short histories would otherwise be cut into one-page
+  // pieces whose merges cost more than the pages (measured on the 4K-token workload)
+  const int Geff = (int)min((long long)gridDim.x, (W + kMinPagesPerCta - 1) / kMinPagesPerCta);
   if ((int)blockIdx.x >= Geff) return;
   const long long g_begin = range_begin(blockIdx.x, W, Geff);
   const long long g_end = range_begin(blockIdx.x + 1, W, Geff);
@@ -614,8 +617,7 @@ static helix_status launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const
                            int grid, cudaStream_t stream) {
   const size_t smem = smem_bytes_for<D>(p.units);
   auto kern = gqa_partial_kernel<D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
+  if (allow_max_dynamic_smem(reinterpret_cast<const void*>(kern)) != cudaSuccess)
     return HELIX_ERR_CUDA;
   kern<<<grid, kThreads, smem, stream>>>(tmK, tmV, p);
   return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;

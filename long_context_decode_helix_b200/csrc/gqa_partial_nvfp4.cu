@@ -61,6 +61,7 @@ constexpr int kOffKs = kKcBytes, kOffVc = kKcBytes + kKsBytes, kOffVs = 2 * kKcB
 constexpr int kStageBytes = 2 * (kKcBytes + kKsBytes);  // 9216
 constexpr int kRec = kRows * (kD + 3);                  // workspace record: O, m, (unused), lb
 constexpr float kLazy = 8.f;  // base-2 headroom before the reference maximum moves
+constexpr int kMinPagesPerCta = 4;
 constexpr uint32_t kOnes = 0x3C003C00u;  // f16x2 (1, 1)
 
 struct Tail {
@@ -183,7 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
     if (p.o_out != nullptr)
       fused_group_combine(p, bk, &tail->gflag, [] { __syncthreads(); }, tid, warp, lane, kWarps);
   }
-  const int Geff = (int)min((long long)gridDim.x, W);
+  // at least kMinPagesPerCta pages per CTA: short histories would otherwise be cut into one-page
+  // pieces whose merges cost more than the pages (measured on the 4K-token workload)
+  const int Geff = (int)min((long long)gridDim.x, (W + kMinPagesPerCta - 1) / kMinPagesPerCta);
   if ((int)blockIdx.x >= Geff) return;
   const long long g_begin = range_begin(blockIdx.x, W, Geff);
   const long long g_end = range_begin(blockIdx.x + 1, W, Geff);
@@ -618,8 +621,8 @@ size_t gqa_nvfp4_segment_record_floats() { return kRec; }
 helix_status gqa_partial_nvfp4_launch(const GqaParams& p, int grid, cudaStream_t stream) {
   if (p.D != kD) return HELIX_ERR_UNSUPPORTED;
   const size_t smem = gqa_nvfp4_smem_bytes(p.units);
-  if (cudaFuncSetAttribute(gqa_partial_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  if (allow_max_dynamic_smem(reinterpret_cast<const void*>(gqa_partial_nvfp4_kernel)) !=
+      cudaSuccess)
     return HELIX_ERR_CUDA;
   gqa_partial_nvfp4_kernel<<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;

@@ -79,6 +79,9 @@ struct AppendParams {
 };
 helix_status append_launch(const AppendParams& p, cudaStream_t stream);
 
+// Raises a kernel's dynamic shared-memory limit to the device maximum, once per (kernel, device).
+cudaError_t allow_max_dynamic_smem(const void* func);
+
 // rows = B * Hq (the shard stride of o_partial / lse); combines rows [row0, row0 + nrows)
 helix_status combine_launch(int kvp, int rows, int row0, int nrows, int v_dim,
                             const float* o_partial, const float* lse, void* o_out, int o_dtype,

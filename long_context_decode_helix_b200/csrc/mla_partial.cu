@@ -845,8 +845,7 @@ size_t mla_segment_record_floats() { return kRec; }
 helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmQ,
                                 const MlaParams& p, int grid, cudaStream_t stream) {
   const size_t smem = mla_partial_smem_bytes(p.units);
-  if (cudaFuncSetAttribute(mla_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  if (allow_max_dynamic_smem(reinterpret_cast<const void*>(mla_partial_kernel)) != cudaSuccess)
     return HELIX_ERR_CUDA;
   mla_partial_kernel<<<grid, kThreads, smem, stream>>>(tmC, tmQ, p);
   return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
