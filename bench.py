@@ -118,6 +118,15 @@ class ClockSampler:
                  "-lms", "100", "-i", str(self.gpu)], stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # nvidia-smi takes a while to print its first line: wait for it (bounded), so that even a
+        # short timed region falls inside the sampled window
+        t_end = time.time() + 5.0
+        while time.time() < t_end and self.proc.poll() is None:
+            self.fh.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -341,7 +350,6 @@ def run_helix(args):
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
-    time.sleep(0.3)
     torch.cuda.nvtx.range_push("timed_steps")
     start.record(stream)
     for i in range(K):

@@ -59,12 +59,14 @@ constexpr int kChunks = 5;                 // 64-column chunks of a latent row p
 constexpr int kKSteps = 18;                // 288 / 16
 constexpr int kNS = 2;                     // tile stages
 constexpr int kNX = 1;                     // score-exchange buffers (the groups take turns)
+constexpr int kPrefetch = 3;               // tiles fetched into L2 ahead of the TMA loads
 constexpr int kStageBytes = kTok * kChunks * 128;     // 40 KiB
 constexpr int kQBytes = kHeads * kChunks * 128;        // 80 KiB
 constexpr int kSBuf = 2;                               // score-tile buffers in TMEM
 constexpr uint32_t kSCol = 256, kPCol = 384;           // TMEM columns: O [0,256), S 2x64, P 2x32
-constexpr int kXStride = kTok + 4;                     // padded fp32 row of the exchange buffer
-constexpr int kXBytes = kHeads * kXStride * 4;         // 34 KiB
+// exchange buffer: [kTok / 4][kHeads] groups of four fp32 scores, so that the 32 rows of a warp
+// write (remotely) and read 512 contiguous bytes per instruction
+constexpr int kXBytes = kHeads * kTok * 4;             // 32 KiB
 // warps 0-7: two softmax groups of four (group g takes the tiles i with i % 2 == g)
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 10 * 32;
@@ -287,8 +289,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* q_s = smem;                                   // [5 chunks][128 rows][128 B]
   uint8_t* stage_s = q_s + kQBytes;                      // [kNS][5 chunks][64 rows][128 B]
-  float* x_s = reinterpret_cast<float*>(stage_s + kNS * kStageBytes);  // [kNX][128][kXStride]
-  MlaTail* tail = reinterpret_cast<MlaTail*>(x_s + kNX * kHeads * kXStride);
+  float* x_s = reinterpret_cast<float*>(stage_s + kNS * kStageBytes);  // [kNX][kTok/4][128][4]
+  MlaTail* tail = reinterpret_cast<MlaTail*>(x_s + kNX * kHeads * kTok);
   int* pre = reinterpret_cast<int*>(tail + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -403,8 +405,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int u = u_first, cur = -1, qcount = 0;
       int stage = 0;
       uint32_t round = 0;
+      // L2 prefetch kPrefetch tiles ahead of the stage ring: the ring holds only kNS tiles, so
+      // without it each TMA load would wait a full HBM latency behind the tile two steps back.
+      int u_pf = u_first;
+      long long g_pf = g_begin;
+      auto prefetch_upto = [&](long long g_stop) {
+        for (; g_pf < g_stop && g_pf < g_end; ++g_pf) {
+          while (pre[u_pf + 1] <= g_pf) ++u_pf;
+          const int s_ = (u_pf + p.u0) % p.kvp, b_ = (u_pf + p.u0) / p.kvp;
+          const int pg = __ldg(p.page_table + ((size_t)s_ * p.B + b_) * p.max_pages +
+                               (int)(g_pf - pre[u_pf]));
+          if (pg < 0 || pg >= p.num_pages) continue;
+          for (int c = 0; c < kChunks; ++c)
+            tma_prefetch_l2_2d(&tmC, (4 * rank + c) * 64, pg * kPageTok);
+        }
+      };
       for (long long g = g_begin; g < g_end; ++g) {
         if (*(volatile int*)&tail->abort_) break;
+        prefetch_upto(g + kPrefetch);
         while (pre[u + 1] <= g) ++u;
         const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
         if (u != cur) {  // (re)load this CTA's half of q for request b
@@ -420,13 +438,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           cur = u;
           ++qcount;
         }
+        // the page id is read before the wait for the stage, so its latency overlaps the wait
+        const int lt = (int)(g - pre[u]);  // tile within the unit
+        const int page = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + lt);
         if (round > 0 && !mbar_wait(&tail->stage_empty[stage], (round - 1) & 1)) {
           raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
           *(volatile int*)&tail->abort_ = 1;
           break;
         }
-        const int lt = (int)(g - pre[u]);  // tile within the unit
-        const int page = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + lt);
         if (page < 0 || page >= p.num_pages) {
           raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
           tail->stage_ok[stage] = 0;
@@ -615,10 +634,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // the one exchange buffer serves the tiles in turn: tile i-1's scores must have been read
       if (i >= 1) wwait(&tail->x_free[0], (uint32_t)((i - 1) & 1), true);
       {
-        const uint32_t dst = x_peer + (uint32_t)(h * kXStride * 4);
+        const uint32_t dst = x_peer + (uint32_t)(h * 16);
 #pragma unroll
         for (int c = 0; c < kTok; c += 4)
-          st_async_v4(dst + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3], xfull_peer);
+          st_async_v4(dst + (c / 4) * kHeads * 16, sv[c], sv[c + 1], sv[c + 2], sv[c + 3],
+                      xfull_peer);
       }
       // the previous tile closed a segment owned by the other group: join its flush before this
       // tile's P can reach the MMA (its P V would overwrite O)
@@ -626,10 +646,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ---- B: add the peer's partial, softmax, P into TMEM ----
       wwait(&tail->x_full[0], (uint32_t)(i & 1), true);
       {
-        const float* mine = x_s + (size_t)h * kXStride;
+        const float* mine = x_s + (size_t)h * 4;
 #pragma unroll
         for (int c = 0; c < kTok; c += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(mine + c);
+          const float4 v = *reinterpret_cast<const float4*>(mine + (c / 4) * kHeads * 4);
           sv[c] += v.x;
           sv[c + 1] += v.y;
           sv[c + 2] += v.z;
