@@ -57,6 +57,8 @@ constexpr int kTok = 64;                   // tokens per tile (one page)
 constexpr int kPageTok = 64;               // tokens per page
 constexpr int kChunks = 5;                 // 64-column chunks of a latent row per CTA
 constexpr int kKSteps = 18;                // 288 / 16
+constexpr int kSPart = 9;                  // score k-steps issued between looks at P V
+static_assert(kKSteps % kSPart == 0, "score tile issued in equal parts");
 constexpr int kNS = 2;                     // tile stages
 constexpr int kNX = 1;                     // score-exchange buffers (the groups take turns)
 constexpr int kPrefetch = 3;               // tiles fetched into L2 ahead of the TMA loads
@@ -471,6 +473,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr uint32_t idPV = make_idesc(128, kHalfDV, true);
       const long long n = g_end - g_begin;
       long long ns = 0, npv = 0;
+      int s_k = 0;  // k-steps of S(ns) issued so far
       int u_s = u_first, u_pv = u_first, cur = -1, qcount = 0;
       bool dead = false;
       uint64_t t_last = 0;
@@ -506,35 +509,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (ns < n) {
           const long long g = g_begin + ns;
-          while (pre[u_s + 1] <= g) ++u_s;
-          if (u_s != cur && mbar_test(&tail->q_full, qcount & 1)) {  // this unit's q has landed
-            cur = u_s;
-            ++qcount;
-          }
           const int st = (int)(ns % kNS), sb = (int)(ns % kSBuf);
-          if (u_s == cur && mbar_test(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) &&
-              (ns < kSBuf ||
-               mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - kSBuf) / kSBuf) & 1)))) {
-            tc_fence_after();
-            // S_partial = q[:, half] C_tile[:, half]^T: 18 k-steps of 16 over this CTA's columns
-            // Descriptors are built once per tile; a k-step only advances the start address
-            // (16-byte units): 32 B inside a 128-byte swizzle row, one chunk (q: 16 KiB, tile:
-            // 4 KiB) per 4 k-steps. This CTA's columns start 32 * rank elements into its chunks.
+          bool go = s_k > 0;  // a started score tile goes on without further checks
+          if (!go) {
+            while (pre[u_s + 1] <= g) ++u_s;
+            if (u_s != cur && mbar_test(&tail->q_full, qcount & 1)) {  // this unit's q has landed
+              cur = u_s;
+              ++qcount;
+            }
+            go = u_s == cur && mbar_test(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) &&
+                 (ns < kSBuf ||
+                  mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - kSBuf) / kSBuf) & 1)));
+            if (go) tc_fence_after();
+          }
+          if (go) {
+            // S_partial = q[:, half] C_tile[:, half]^T: 18 k-steps of 16 over this CTA's columns,
+            // kSPart at a time, so that a P V product that becomes ready meanwhile goes out
+            // between the parts instead of behind the whole tile. A k-step only advances the
+            // start address (16-byte units): 32 B inside a 128-byte swizzle row, one chunk (q:
+            // 16 KiB, tile: 8 KiB) per 4 k-steps. This CTA's columns start 32 * rank elements
+            // into its chunks.
             const uint64_t a0 = smem_desc(qbase, 16, 1024, kSwizzle128);
             const uint64_t b0 = smem_desc(smem_u32(stage_s + st * kStageBytes), 16, 1024,
                                           kSwizzle128);
             const uint32_t d_s = tmem + kSCol + sb * kTok;
 #pragma unroll
-            for (int ks = 0; ks < kKSteps; ++ks) {
+            for (int j = 0; j < kSPart; ++j) {
+              const int ks = s_k + j;
               const uint32_t kk = (uint32_t)ks + 2u * rank;  // 16-element step inside the chunks
               const uint32_t ch = kk >> 2, in_row = (kk & 3u) * 2u;
               tc_mma(d_s, a0 + ch * (kHeads * 128 / 16) + in_row,
                      b0 + ch * (kTok * 128 / 16) + in_row, idS, ks > 0);
             }
-            tc_commit(&tail->s_full[sb]);
-            // the last tile of a unit (or of the range) releases q for the next unit
-            if (g + 1 == g_end || g + 1 == pre[u_s + 1]) tc_commit(&tail->q_empty);
-            ++ns;
+            s_k += kSPart;
+            if (s_k == kKSteps) {
+              tc_commit(&tail->s_full[sb]);
+              // the last tile of a unit (or of the range) releases q for the next unit
+              if (g + 1 == g_end || g + 1 == pre[u_s + 1]) tc_commit(&tail->q_empty);
+              s_k = 0;
+              ++ns;
+            }
             progress = true;
           }
         }
@@ -681,11 +695,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 4; ++c) t[c] = fmaxf(t[c], t[c + 4]);
         mx = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
       }
-      // V rows past the end of the history are zeroed before the P V product reads them
-      if (nvalid < kTok && !dead) {
+      // V rows past the end of the history, or all of a tile whose page id is out of range (not
+      // loaded: stale or never-written shared memory), are zeroed before the P V product reads
+      // them, since a zero weight times a non-finite value is not zero
+      const int keep = tile_ok ? nvalid : 0;
+      if (keep < kTok && !dead) {
         uint8_t* stg = stage_s + st_i * kStageBytes;
-        for (int e = h; e < (kTok - nvalid) * 4 * 8; e += kHeads) {
-          const int row = nvalid + e / 32, rem = e % 32;
+        for (int e = h; e < (kTok - keep) * 4 * 8; e += kHeads) {
+          const int row = keep + e / 32, rem = e % 32;
           *reinterpret_cast<uint4*>(stg + (rem / 8) * kTok * 128 + row * 128 + (rem % 8) * 16) =
               make_uint4(0, 0, 0, 0);
         }

@@ -117,3 +117,25 @@ def test_mla_full_1m_sampled():
         del C
     del cache
     torch.cuda.empty_cache()
+
+
+def test_mla_bad_page_id_sets_error_and_skips():
+    """A page id outside the pool sets the device error bit, and that page's 64 tokens are left out
+    of its shard (masked scores, zeroed values); the rest of the shard is attended exactly."""
+    w = MLA.with_(B=1, S=640, kvp=2)
+    cache = _gpu.make_cache(w)
+    _gpu.fill(cache, w, [640])
+    cache.page_table[1, 0, 2] = 10 ** 6  # beyond the pool: local tokens 128..191 of shard 1
+    cache.clear_errors()
+    q = wl.query(w, "cuda")
+    o_part, lse_part, _, _ = _run(cache, w, q)
+    assert cache.err_bits() & _gpu.hx().DEVERR_PAGE_ID
+    assert np.isfinite(o_part).all() and np.isfinite(lse_part).all()
+    C = oracle.attention._f64(wl.kv_range_bf16(w, "c", 0, 0, 0, 640, "cuda"))
+    qb = oracle.attention._f64(q[0])
+    sets = _gpu.shard_sets(w, 640)
+    kept = np.concatenate([sets[1][:128], sets[1][192:]])
+    for s_, idx in ((0, sets[0]), (1, kept)):
+        Os, Ls = oracle.attend(qb, C[idx], C[idx][:, : w.dv], w.softmax_scale)
+        _gpu.assert_close_O(o_part[s_, 0], Os, f"O_partial s={s_}")
+        _gpu.assert_close_lse(lse_part[s_, 0], Ls, f"lse_partial s={s_}")
