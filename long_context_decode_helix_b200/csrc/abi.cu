@@ -310,6 +310,7 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
     m.shard_lens = c->shard_lens;
     m.o_part = o_partial;
     m.lse = lse;
+    m.q = static_cast<const uint16_t*>(q);
     m.tickets = reinterpret_cast<int32_t*>(workspace);
     m.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes +
                                      plan.gticket_bytes);

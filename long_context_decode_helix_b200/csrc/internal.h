@@ -50,6 +50,7 @@ struct MlaParams {
   const int32_t* shard_lens;  // [kvp][B]
   float* o_part;              // [kvp][B][128][512]
   float* lse;                 // [kvp][B][128]
+  const uint16_t* q;          // bf16 [B][128][576] (also read through the q tensor map)
   int32_t* tickets;           // [units][2], zero between launches
   float* seg;                 // [clusters][2 slots][2 halves][record]
   uint32_t* err;              // may be null

@@ -12,11 +12,13 @@
 // Sizes force a two-CTA design. O for 128 heads x 512 columns in fp32 fills all 512 TMEM columns
 // and q (128 x 576 bf16) alone is 144 KiB, so one CTA cannot hold q, a score tile and O. A cluster
 // of two CTAs works on the same 64-token tiles (one page each):
-//   * CTA r keeps half of q's contraction (head-dim elements [288 r, 288 r + 288)) in shared memory
-//     and computes a partial score tile S_r = q[:, half] C[:, half]^T (M = 128 heads, N = 64 tokens,
-//     K = 288) into TMEM. A tcgen05.mma of M = 128 costs about the same for any N up to 128
-//     (measured: about 110 SM cycles for one K = 16 step), so the score tile is as wide as the
-//     shared-memory budget allows;
+//   * CTA r takes half of the contraction, head-dim elements [288 r, 288 r + 288): four whole
+//     64-column chunks of q in shared memory (chunks 0-3, or 5-8) and its 32 columns of the
+//     shared chunk 4 in 16 TMEM columns (loaded by the softmax warps at each new request), and
+//     computes a partial score tile S_r = q[:, half] C[:, half]^T (M = 128 heads, N = 64 tokens,
+//     K = 288) into TMEM: 2 k-steps with A from TMEM, then 16 with both operands in shared memory.
+//     A tcgen05.mma of M = 128 costs about the same for any N up to 128 (measured: about 110 SM
+//     cycles for one K = 16 step), so the score tile is as wide as a page;
 //   * the two CTAs swap their partials through distributed shared memory: st.async stores into the
 //     peer's exchange buffer complete a transaction count on the peer's mbarrier, and the buffer is
 //     handed back with a relaxed remote arrive (no multicast loads anywhere), so both hold the same
@@ -26,7 +28,10 @@
 //     TS form of the MMA (A = P from TMEM, B = V read straight from the latent tile it already holds,
 //     MN-major).
 // Each CTA loads five 64-column chunks of every latent row (chunks 0-4 or 4-8), so together the pair
-// reads the 576-wide row once plus one 64-column chunk.
+// reads the 576-wide row once plus one 64-column chunk. With q's half chunk in TMEM, three 40 KiB
+// tile stages fit beside q (64 KiB) and the exchange buffer: the load of a tile waits for the P V
+// product three tiles back, which is what bounds the tile period (the chain of one tile: load,
+// scores, exchange, softmax, P V, over the number of stages).
 //
 // Warps: 0-7 softmax / epilogue in two groups of four (group g takes the tiles i with i % 2 == g,
 // so two tiles are in the softmax at once; thread h of a group owns head h = TMEM lane h), 8 TMA
@@ -56,16 +61,19 @@ constexpr int kDV = 512, kHalfDV = 256;  // V: the first 512 of the 576 latent c
 constexpr int kTok = 64;                   // tokens per tile (one page)
 constexpr int kPageTok = 64;               // tokens per page
 constexpr int kChunks = 5;                 // 64-column chunks of a latent row per CTA
-constexpr int kKSteps = 18;                // 288 / 16
-constexpr int kSPart = 9;                  // score k-steps issued between looks at P V
-static_assert(kKSteps % kSPart == 0, "score tile issued in equal parts");
-constexpr int kNS = 2;                     // tile stages
+constexpr int kQChunks = 4;                // full 64-column chunks of q per CTA (in shared memory)
+constexpr int kKSteps = 18;                // 288 / 16: 2 over the half chunk, 16 over whole ones
+static_assert(2 + 4 * kQChunks == kKSteps, "a CTA's 288 columns: four chunks and a half");
+constexpr int kNS = 3;                     // tile stages
 constexpr int kNX = 1;                     // score-exchange buffers (the groups take turns)
 constexpr int kPrefetch = 3;               // tiles fetched into L2 ahead of the TMA loads
 constexpr int kStageBytes = kTok * kChunks * 128;     // 40 KiB
-constexpr int kQBytes = kHeads * kChunks * 128;        // 80 KiB
+constexpr int kQBytes = kHeads * kQChunks * 128;       // 64 KiB
 constexpr int kSBuf = 2;                               // score-tile buffers in TMEM
 constexpr uint32_t kSCol = 256, kPCol = 384;           // TMEM columns: O [0,256), S 2x64, P 2x32
+// and q's 32 columns of the shared chunk (the half of columns 256..319 this CTA takes), 16 columns
+// of bf16 pairs: the A operand of the two score k-steps over that half chunk
+constexpr uint32_t kQhCol = 448;
 // exchange buffer: [kTok / 4][kHeads] groups of four fp32 scores, so that the 32 rows of a warp
 // write (remotely) and read 512 contiguous bytes per instruction
 constexpr int kXBytes = kHeads * kTok * 4;             // 32 KiB
@@ -81,6 +89,7 @@ struct MlaTail {
   uint64_t p_full[2], p_empty[2];
   uint64_t x_full[kNX], x_free[kNX];
   uint64_t q_full, q_empty;
+  uint64_t qh_full;  // q's half chunk for the next unit is in TMEM (one arrival per warp of a group)
   int stage_ok[kNS];
   uint64_t m_ready[2][4];   // [publishing group][32-row slice]: mpub holds its latest maximum
   uint64_t seg_ready;       // segment end: the non-owning group has stored its (m, l)
@@ -242,6 +251,16 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+// 16 consecutive 32-bit columns of this thread's TMEM lane (raw bits)
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -289,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* q_s = smem;                                   // [5 chunks][128 rows][128 B]
+  uint8_t* q_s = smem;                                   // [4 chunks][128 rows][128 B]
   uint8_t* stage_s = q_s + kQBytes;                      // [kNS][5 chunks][64 rows][128 B]
   float* x_s = reinterpret_cast<float*>(stage_s + kNS * kStageBytes);  // [kNX][kTok/4][128][4]
   MlaTail* tail = reinterpret_cast<MlaTail*>(x_s + kNX * kHeads * kTok);
@@ -336,6 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(&tail->q_full, 1);
     mbar_init(&tail->q_empty, 1);
+    mbar_init(&tail->qh_full, 4);
     tail->flag = 0;
     tail->abort_ = 0;
     fence_mbar_init();
@@ -433,9 +453,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             *(volatile int*)&tail->abort_ = 1;
             break;
           }
+          // the four chunks of q this CTA takes whole: 0-3 (r = 0) or 5-8 (r = 1); its half of
+          // chunk 4 goes to TMEM (loaded by the softmax warps)
           mbar_arrive_expect_tx(&tail->q_full, kQBytes);
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_2d(q_s + c * kHeads * 128, &tmQ, (4 * rank + c) * 64, b * kHeads,
+          for (int c = 0; c < kQChunks; ++c)
+            tma_load_2d(q_s + c * kHeads * 128, &tmQ, (c + 5 * rank) * 64, b * kHeads,
                         &tail->q_full);
           cur = u;
           ++qcount;
@@ -473,7 +495,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr uint32_t idPV = make_idesc(128, kHalfDV, true);
       const long long n = g_end - g_begin;
       long long ns = 0, npv = 0;
-      int s_k = 0;  // k-steps of S(ns) issued so far
       int u_s = u_first, u_pv = u_first, cur = -1, qcount = 0;
       bool dead = false;
       uint64_t t_last = 0;
@@ -509,46 +530,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (ns < n) {
           const long long g = g_begin + ns;
-          const int st = (int)(ns % kNS), sb = (int)(ns % kSBuf);
-          bool go = s_k > 0;  // a started score tile goes on without further checks
-          if (!go) {
-            while (pre[u_s + 1] <= g) ++u_s;
-            if (u_s != cur && mbar_test(&tail->q_full, qcount & 1)) {  // this unit's q has landed
-              cur = u_s;
-              ++qcount;
-            }
-            go = u_s == cur && mbar_test(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) &&
-                 (ns < kSBuf ||
-                  mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - kSBuf) / kSBuf) & 1)));
-            if (go) tc_fence_after();
+          while (pre[u_s + 1] <= g) ++u_s;
+          if (u_s != cur && mbar_test(&tail->q_full, qcount & 1) &&
+              mbar_test(&tail->qh_full, qcount & 1)) {  // this unit's q has landed (both parts)
+            cur = u_s;
+            ++qcount;
           }
-          if (go) {
-            // S_partial = q[:, half] C_tile[:, half]^T: 18 k-steps of 16 over this CTA's columns,
-            // kSPart at a time, so that a P V product that becomes ready meanwhile goes out
-            // between the parts instead of behind the whole tile. A k-step only advances the
-            // start address (16-byte units): 32 B inside a 128-byte swizzle row, one chunk (q:
-            // 16 KiB, tile: 8 KiB) per 4 k-steps. This CTA's columns start 32 * rank elements
-            // into its chunks.
+          const int st = (int)(ns % kNS), sb = (int)(ns % kSBuf);
+          if (u_s == cur && mbar_test(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) &&
+              (ns < kSBuf ||
+               mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - kSBuf) / kSBuf) & 1)))) {
+            tc_fence_after();
+            // S_partial = q[:, cols] C_tile[:, cols]^T over this CTA's 288 columns, 18 k-steps of
+            // 16 issued back to back (breaking them up to let a ready P V product through costs
+            // more than it gains). The two k-steps over the half chunk (A = q's 32 columns from
+            // TMEM) go first, next to the P V product (also A from TMEM) that usually precedes
+            // them: the tensor pipe loses time at each switch between shared-memory and
+            // tensor-memory A operands. A k-step only advances the start address (16-byte units):
+            // 32 B inside a 128-byte swizzle row, one chunk (q: 16 KiB, tile: 8 KiB) per 4 k-steps.
             const uint64_t a0 = smem_desc(qbase, 16, 1024, kSwizzle128);
             const uint64_t b0 = smem_desc(smem_u32(stage_s + st * kStageBytes), 16, 1024,
                                           kSwizzle128);
             const uint32_t d_s = tmem + kSCol + sb * kTok;
 #pragma unroll
-            for (int j = 0; j < kSPart; ++j) {
-              const int ks = s_k + j;
-              const uint32_t kk = (uint32_t)ks + 2u * rank;  // 16-element step inside the chunks
-              const uint32_t ch = kk >> 2, in_row = (kk & 3u) * 2u;
+            for (int hj = 0; hj < 2; ++hj)  // B = this CTA's 32 columns of tile chunk 4
+              tc_mma_ts(d_s, tmem + kQhCol + (uint32_t)hj * 8,
+                        b0 + 4u * (1u - rank) * (kTok * 128 / 16) + 2u * ((uint32_t)hj + 2u * rank),
+                        idS, hj > 0);
+#pragma unroll
+            for (int f = 0; f < 4 * kQChunks; ++f) {  // q's whole chunks, tile chunks r .. r + 3
+              const uint32_t ch = (uint32_t)f >> 2, in_row = ((uint32_t)f & 3u) * 2u;
               tc_mma(d_s, a0 + ch * (kHeads * 128 / 16) + in_row,
-                     b0 + ch * (kTok * 128 / 16) + in_row, idS, ks > 0);
+                     b0 + (ch + rank) * (kTok * 128 / 16) + in_row, idS, true);
             }
-            s_k += kSPart;
-            if (s_k == kKSteps) {
-              tc_commit(&tail->s_full[sb]);
-              // the last tile of a unit (or of the range) releases q for the next unit
-              if (g + 1 == g_end || g + 1 == pre[u_s + 1]) tc_commit(&tail->q_empty);
-              s_k = 0;
-              ++ns;
-            }
+            tc_commit(&tail->s_full[sb]);
+            // the last tile of a unit (or of the range) releases q for the next unit
+            if (g + 1 == g_end || g + 1 == pre[u_s + 1]) tc_commit(&tail->q_empty);
+            ++ns;
             progress = true;
           }
         }
@@ -618,6 +636,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       m_own = -INFINITY;
       l_own = 0.f;
     };
+    // q's half chunk (this CTA's 32 of columns 256..319) of request bq into this thread's TMEM
+    // lane: the A operand of the score k-steps over that chunk. A group loads it for the next
+    // unit once it has read the scores of the unit's last tile (all of the unit's score MMAs have
+    // then completed), and arrives on qh_full whether or not it could.
+    auto load_q_half = [&](int bq) {
+      if (!dead) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.q + ((size_t)bq * kHeads + h) * 576 + 256 + 32 * rank);
+        uint32_t v[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 x = __ldg(src + c);
+          v[4 * c] = x.x;
+          v[4 * c + 1] = x.y;
+          v[4 * c + 2] = x.z;
+          v[4 * c + 3] = x.w;
+        }
+        tmem_st16u(tl + kQhCol, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->qh_full);
+    };
+    if (grp == 0 && active) load_q_half((u_first + p.u0) / p.kvp);
     float sv[kTok];
     for (long long i = grp; i < n_tiles; i += 2) {
       const long long g = g_begin + i;
@@ -645,6 +687,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->s_empty[sb]);
+      if (seg_end && g + 1 < g_end) {  // the next tile starts a new unit: its q half chunk
+        int un = u;
+        while (pre[un + 1] <= g + 1) ++un;
+        load_q_half((un + p.u0) / p.kvp);
+      }
       // the one exchange buffer serves the tiles in turn: tile i-1's scores must have been read
       if (i >= 1) wwait(&tail->x_free[0], (uint32_t)((i - 1) & 1), true);
       {
