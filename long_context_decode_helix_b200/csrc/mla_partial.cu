@@ -35,8 +35,9 @@
 //
 // Warps: 0-7 softmax / epilogue in two groups of four (group g takes the tiles i with i % 2 == g,
 // so two tiles are in the softmax at once; thread h of a group owns head h = TMEM lane h), 8 TMA
-// producer, 9 MMA issuer (one elected thread, which issues whichever of the next S tile or the next
-// P V product is ready) and TMEM allocator. Each group has its own TMEM score buffer, so the tensor
+// producer (and L2 prefetch one tile ahead), 9 score-MMA issuer and TMEM allocator, 10 P V issuer
+// (one thread each, so a ready P V never waits behind a score tile). Each group has its own TMEM
+// score buffer, so the tensor
 // core computes the next tile's scores while a group works on its tile. The groups share one reference maximum per head, handed from the owner
 // of tile i-1 to the owner of tile i through shared memory and a named barrier; each group keeps its
 // own running sum, and the two are merged at the end of a segment. O is rescaled lazily: the exponent base only moves when
@@ -66,7 +67,7 @@ constexpr int kKSteps = 18;                // 288 / 16: 2 over the half chunk, 1
 static_assert(2 + 4 * kQChunks == kKSteps, "a CTA's 288 columns: four chunks and a half");
 constexpr int kNS = 3;                     // tile stages
 constexpr int kNX = 1;                     // score-exchange buffers (the groups take turns)
-constexpr int kPrefetch = 3;               // tiles fetched into L2 ahead of the TMA loads
+constexpr int kPrefetch = 1;               // tiles fetched into L2 ahead of the TMA loads
 constexpr int kStageBytes = kTok * kChunks * 128;     // 40 KiB
 constexpr int kQBytes = kHeads * kQChunks * 128;       // 64 KiB
 constexpr int kSBuf = 2;                               // score-tile buffers in TMEM
@@ -78,8 +79,8 @@ constexpr uint32_t kQhCol = 448;
 // write (remotely) and read 512 contiguous bytes per instruction
 constexpr int kXBytes = kHeads * kTok * 4;             // 32 KiB
 // warps 0-7: two softmax groups of four (group g takes the tiles i with i % 2 == g)
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 10 * 32;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kPvWarp = 10;
+constexpr int kThreads = 11 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRec = kHeads * (kHalfDV + 3);           // floats per segment record (one half)
 
@@ -487,101 +488,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    // ====================================== MMA issuer =========================================
+    // ================================== score MMA issuer =======================================
+    // S(i) goes out as soon as its tile has landed, its TMEM score buffer is free and its unit's
+    // q is in place; the P V products have their own issuing thread (below), so a ready P V never
+    // waits behind the 18 score MMAs of the next tile. Each thread's commits track only its own
+    // MMAs, and the two write different accumulators.
     if (lane == 0 && active) {
-      // Event-driven issue: the next score tile S(ns) goes out as soon as its stage has landed and
-      // its TMEM buffer is free, independent of the P V products, which follow the softmax.
       constexpr uint32_t idS = make_idesc(128, kTok, false);
+      const long long n = g_end - g_begin;
+      int u_s = u_first, cur = -1, qcount = 0;
+      bool dead = false;
+      const uint32_t qbase = smem_u32(q_s);
+      for (long long ns = 0; ns < n; ++ns) {
+        const long long g = g_begin + ns;
+        if (*(volatile int*)&tail->abort_) break;
+        while (pre[u_s + 1] <= g) ++u_s;
+        if (u_s != cur) {  // this unit's q: the shared-memory chunks and the TMEM half chunk
+          if (!mbar_wait(&tail->q_full, (uint32_t)(qcount & 1)) ||
+              !mbar_wait(&tail->qh_full, (uint32_t)(qcount & 1))) {
+            dead = true;
+            break;
+          }
+          cur = u_s;
+          ++qcount;
+        }
+        const int st = (int)(ns % kNS), sb = (int)(ns % kSBuf);
+        if (!mbar_wait(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) ||
+            (ns >= kSBuf &&
+             !mbar_wait(&tail->s_empty[sb], (uint32_t)(((ns - kSBuf) / kSBuf) & 1)))) {
+          dead = true;
+          break;
+        }
+        tc_fence_after();
+        // S_partial = q[:, cols] C_tile[:, cols]^T over this CTA's 288 columns, 18 k-steps of 16
+        // issued back to back. The two k-steps over the half chunk (A = q's 32 columns from TMEM)
+        // go first: the tensor pipe loses time at each switch between shared-memory and
+        // tensor-memory A operands, and the P V product before them also reads A from TMEM. A
+        // k-step only advances the start address (16-byte units): 32 B inside a 128-byte swizzle
+        // row, one chunk (q: 16 KiB, tile: 8 KiB) per 4 k-steps.
+        const uint64_t a0 = smem_desc(qbase, 16, 1024, kSwizzle128);
+        const uint64_t b0 = smem_desc(smem_u32(stage_s + st * kStageBytes), 16, 1024,
+                                      kSwizzle128);
+        const uint32_t d_s = tmem + kSCol + sb * kTok;
+#pragma unroll
+        for (int hj = 0; hj < 2; ++hj)  // B = this CTA's 32 columns of tile chunk 4
+          tc_mma_ts(d_s, tmem + kQhCol + (uint32_t)hj * 8,
+                    b0 + 4u * (1u - rank) * (kTok * 128 / 16) + 2u * ((uint32_t)hj + 2u * rank),
+                    idS, hj > 0);
+#pragma unroll
+        for (int f = 0; f < 4 * kQChunks; ++f) {  // q's whole chunks, tile chunks r .. r + 3
+          const uint32_t ch = (uint32_t)f >> 2, in_row = ((uint32_t)f & 3u) * 2u;
+          tc_mma(d_s, a0 + ch * (kHeads * 128 / 16) + in_row,
+                 b0 + (ch + rank) * (kTok * 128 / 16) + in_row, idS, true);
+        }
+        tc_commit(&tail->s_full[sb]);
+        // the last tile of a unit (or of the range) releases q for the next unit
+        if (g + 1 == g_end || g + 1 == pre[u_s + 1]) tc_commit(&tail->q_empty);
+      }
+      if (dead) {
+        raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
+        *(volatile int*)&tail->abort_ = 1;
+      }
+    }
+  } else if (warp == kPvWarp) {
+    // ==================================== P V issuer ==========================================
+    // O += P V for each tile in order, as soon as its P is in TMEM; completing it frees the tile
+    // stage (its scores were done before P existed) and the group's P buffer.
+    if (lane == 0 && active) {
       constexpr uint32_t idPV = make_idesc(128, kHalfDV, true);
       const long long n = g_end - g_begin;
-      long long ns = 0, npv = 0;
-      int u_s = u_first, u_pv = u_first, cur = -1, qcount = 0;
+      int u_pv = u_first;
       bool dead = false;
-      uint64_t t_last = 0;
-      int idle = 0;
-      const uint32_t qbase = smem_u32(q_s);
-      while (npv < n && !dead) {
-        bool progress = false;
-        // P V first: it is on the critical path (it frees the tile's stage and the P buffer)
-        if (npv < ns) {
-          const int pb = (int)(npv & 1);
-          if (mbar_test(&tail->p_full[pb], (uint32_t)((npv >> 1) & 1))) {
-            const long long g = g_begin + npv;
-            while (pre[u_pv + 1] <= g) ++u_pv;
-            const bool fresh = g == g_begin || g == pre[u_pv];  // first tile of a segment
-            const int st = (int)(npv % kNS);
-            tc_fence_after();
-            const uint32_t vbase = smem_u32(stage_s + st * kStageBytes);
-#pragma unroll
-            for (int ks = 0; ks < kTok / 16; ++ks) {
-              // A = P [128 heads x 16 tokens] from TMEM (8 columns per 16 tokens)
-              // B = V [16 tokens x 256 columns], MN-major, 128-byte swizzle: 64-column groups one
-              // 32-row chunk (4 KiB) apart, 8-token groups 1 KiB apart
-              const uint64_t bdesc =
-                  smem_desc(vbase + ks * 16 * 128, kTok * 128, 1024, kSwizzle128);
-              tc_mma_ts(tmem, tmem + kPCol + pb * (kTok / 2) + ks * 8, bdesc, idPV,
-                        !(fresh && ks == 0));
-            }
-            tc_commit(&tail->stage_empty[st]);
-            tc_commit(&tail->p_empty[pb]);
-            ++npv;
-            progress = true;
-          }
+      for (long long npv = 0; npv < n; ++npv) {
+        if (*(volatile int*)&tail->abort_) break;
+        const int pb = (int)(npv & 1);
+        if (!mbar_wait(&tail->p_full[pb], (uint32_t)((npv >> 1) & 1))) {
+          dead = true;
+          break;
         }
-        if (ns < n) {
-          const long long g = g_begin + ns;
-          while (pre[u_s + 1] <= g) ++u_s;
-          if (u_s != cur && mbar_test(&tail->q_full, qcount & 1) &&
-              mbar_test(&tail->qh_full, qcount & 1)) {  // this unit's q has landed (both parts)
-            cur = u_s;
-            ++qcount;
-          }
-          const int st = (int)(ns % kNS), sb = (int)(ns % kSBuf);
-          if (u_s == cur && mbar_test(&tail->stage_full[st], (uint32_t)((ns / kNS) & 1)) &&
-              (ns < kSBuf ||
-               mbar_test(&tail->s_empty[sb], (uint32_t)(((ns - kSBuf) / kSBuf) & 1)))) {
-            tc_fence_after();
-            // S_partial = q[:, cols] C_tile[:, cols]^T over this CTA's 288 columns, 18 k-steps of
-            // 16 issued back to back (breaking them up to let a ready P V product through costs
-            // more than it gains). The two k-steps over the half chunk (A = q's 32 columns from
-            // TMEM) go first, next to the P V product (also A from TMEM) that usually precedes
-            // them: the tensor pipe loses time at each switch between shared-memory and
-            // tensor-memory A operands. A k-step only advances the start address (16-byte units):
-            // 32 B inside a 128-byte swizzle row, one chunk (q: 16 KiB, tile: 8 KiB) per 4 k-steps.
-            const uint64_t a0 = smem_desc(qbase, 16, 1024, kSwizzle128);
-            const uint64_t b0 = smem_desc(smem_u32(stage_s + st * kStageBytes), 16, 1024,
-                                          kSwizzle128);
-            const uint32_t d_s = tmem + kSCol + sb * kTok;
+        const long long g = g_begin + npv;
+        while (pre[u_pv + 1] <= g) ++u_pv;
+        const bool fresh = g == g_begin || g == pre[u_pv];  // first tile of a segment
+        const int st = (int)(npv % kNS);
+        tc_fence_after();
+        const uint32_t vbase = smem_u32(stage_s + st * kStageBytes);
 #pragma unroll
-            for (int hj = 0; hj < 2; ++hj)  // B = this CTA's 32 columns of tile chunk 4
-              tc_mma_ts(d_s, tmem + kQhCol + (uint32_t)hj * 8,
-                        b0 + 4u * (1u - rank) * (kTok * 128 / 16) + 2u * ((uint32_t)hj + 2u * rank),
-                        idS, hj > 0);
-#pragma unroll
-            for (int f = 0; f < 4 * kQChunks; ++f) {  // q's whole chunks, tile chunks r .. r + 3
-              const uint32_t ch = (uint32_t)f >> 2, in_row = ((uint32_t)f & 3u) * 2u;
-              tc_mma(d_s, a0 + ch * (kHeads * 128 / 16) + in_row,
-                     b0 + (ch + rank) * (kTok * 128 / 16) + in_row, idS, true);
-            }
-            tc_commit(&tail->s_full[sb]);
-            // the last tile of a unit (or of the range) releases q for the next unit
-            if (g + 1 == g_end || g + 1 == pre[u_s + 1]) tc_commit(&tail->q_empty);
-            ++ns;
-            progress = true;
-          }
+        for (int ks = 0; ks < kTok / 16; ++ks) {
+          // A = P [128 heads x 16 tokens] from TMEM (8 columns per 16 tokens)
+          // B = V [16 tokens x 256 columns], MN-major, 128-byte swizzle: 64-column groups one
+          // 64-row chunk (8 KiB) apart, 8-token groups 1 KiB apart
+          const uint64_t bdesc = smem_desc(vbase + ks * 16 * 128, kTok * 128, 1024, kSwizzle128);
+          tc_mma_ts(tmem, tmem + kPCol + pb * (kTok / 2) + ks * 8, bdesc, idPV,
+                    !(fresh && ks == 0));
         }
-        // bounded: give up after the wait limit passes without any progress (t_last = 0 means the
-        // clock is not running; it starts on the first batch of 256 idle polls)
-        if (progress) {
-          idle = 0;
-          t_last = 0;
-        } else if (++idle >= 256) {
-          idle = 0;
-          if (*(volatile int*)&tail->abort_) dead = true;
-          const uint64_t now = global_timer_ns();
-          if (t_last == 0) t_last = now;
-          else if (now - t_last > kWaitLimitNs) dead = true;
-        }
+        tc_commit(&tail->stage_empty[st]);
+        tc_commit(&tail->p_empty[pb]);
       }
       if (dead) {
         raise_dev_error(p.err, HELIX_DEVERR_WAIT_TIMEOUT);
