@@ -47,6 +47,8 @@ def parse():
                     help="request groups of the two-stream HOP-B analogue, timed after the main "
                          "steps and reported under 'hopb' (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-read-probe", action="store_true",
+                    help="skip the pure-read bandwidth probe reported beside the roofline")
     ap.add_argument("--cpu-sample-tokens", type=int, default=1 << 19,
                     help="history tokens per sampled head group for the CPU oracle")
     ap.add_argument("--cpu-sample-groups", type=int, default=4)
@@ -158,6 +160,30 @@ class ClockSampler:
 
 
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e data-sheet bandwidth, for context beside the measured peaks
+
+
+def read_probe_gbs(dev, gib: int = 4, reps: int = 5):
+    """HBM read bandwidth of a plain torch reduction over a buffer far larger than L2, best of
+    `reps` (CUDA events): a pure-read figure taken in the same run, for context beside the measured
+    copy peak. It is not one of this library's kernels and runs outside the timed region."""
+    try:
+        x = torch.ones(gib << 28, dtype=torch.float32, device=dev)
+        best = None
+        for _ in range(reps + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.sum(x)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        gbs = x.numel() * 4 / (best * 1e-3) / 1e9
+        del x
+        torch.cuda.empty_cache()
+        return {"gbs": gbs, "how": f"torch.sum over a {gib} GiB fp32 buffer, best of {reps}"}
+    except RuntimeError:
+        return None
 
 
 def measured_peaks():
@@ -434,6 +460,7 @@ def run_helix(args):
                 "gpu_launches": K * 3 * (-(-w.B // per))}
         assert cache.err_bits() == 0, "a HOP-B step reported a device error"
 
+    read_probe = read_probe_gbs(dev) if rank == 0 and not args.no_read_probe else None
     if rank == 0:
         step_bytes = float(np.mean([wl.step_bytes(w, L) for L in lens_at]))
         # the timed kernel: the fused partial + combine (GQA); for MLA the two launches
@@ -451,6 +478,10 @@ def run_helix(args):
                   "frac": achieved_tf / tflops_peak}
         # the binding roof is the one with the longer ideal time
         tensor_bound = flops / (tflops_peak * 1e12) > part_bytes / (peak * 1e9)
+        # context for the HBM roofline: the data-sheet figure and a pure-read probe of this run
+        hbm["frac_of_spec"] = achieved_gbs / SPEC_HBM_GBS
+        if read_probe is not None:
+            hbm["frac_of_read_probe"] = achieved_gbs / read_probe["gbs"]
         roof = dict(tensor if tensor_bound else hbm, bound="tensor" if tensor_bound else "hbm",
                     peak_source=peak_kind, kernel=kname, bytes_per_launch=part_bytes,
                     flops_per_launch=flops, other=(hbm if tensor_bound else tensor),
@@ -470,6 +501,7 @@ def run_helix(args):
             "e2e": e2e,
             "clocks": clk,
             "hopb": hopb,
+            "read_probe": read_probe,
         }
         if not args.no_cpu_baseline and world == 1:
             v, desc, cores, _ = cpu_oracle_sample(w, args.cpu_sample_tokens, args.cpu_sample_groups)

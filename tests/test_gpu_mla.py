@@ -139,3 +139,22 @@ def test_mla_bad_page_id_sets_error_and_skips():
         Os, Ls = oracle.attend(qb, C[idx], C[idx][:, : w.dv], w.softmax_scale)
         _gpu.assert_close_O(o_part[s_, 0], Os, f"O_partial s={s_}")
         _gpu.assert_close_lse(lse_part[s_, 0], Ls, f"lse_partial s={s_}")
+
+
+def test_mla_many_short_units():
+    """Many requests with short, ragged histories: nearly every tile starts a new (request, shard)
+    unit, so q (its shared-memory chunks and its half chunk in TMEM) is reloaded at almost every
+    tile, and many shards are empty. Sharp queries make the weights peaked."""
+    rng = np.random.default_rng(7)
+    lens = [int(x) for x in rng.integers(1, 700, size=12)]
+    lens[3] = 64  # exactly one page in one shard
+    lens[5] = 1
+    w = MLA.with_(B=12, S=max(lens), kvp=8)
+    cache = _gpu.make_cache(w)
+    _gpu.fill(cache, w, lens)
+    assert cache.err_bits() == 0
+    for sharp in (1.0, 8.0):
+        q = wl.query(w, "cuda", scale_by=sharp)
+        res = _run(cache, w, q)
+        assert cache.err_bits() == 0
+        _check(w, q, lens, res, f"many units x{sharp}", heads=list(range(0, 128, 9)))
