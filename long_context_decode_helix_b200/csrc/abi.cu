@@ -112,6 +112,7 @@ helix_status check_cache(const helix_kv_cache* c) {
 struct PartialPlan {
   int grid;
   int units;
+  int max_units;  // units one launch can take (a multiple of the units per request)
   size_t ticket_bytes;
   size_t gticket_bytes;
   size_t seg_bytes;
@@ -129,7 +130,13 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
     int sms = 0, max_smem = 0;
     if (device_sm_count(&sms) != 0 || device_max_smem(&max_smem) != 0) return HELIX_ERR_CUDA;
     plan->units = c->batch * c->kvp;
-    if (mla_partial_smem_bytes(plan->units) > (size_t)max_smem) return HELIX_ERR_CAPACITY;
+    // a launch keeps the prefix sums of its units in shared memory: a batch whose units do not
+    // fit is run as consecutive launches over request ranges
+    if (mla_partial_smem_bytes(0) > (size_t)max_smem) return HELIX_ERR_CAPACITY;
+    const size_t room = ((size_t)max_smem - mla_partial_smem_bytes(0)) / sizeof(int);
+    const int fit = room < (size_t)plan->units ? (int)room : plan->units;
+    plan->max_units = (fit / c->kvp) * c->kvp;
+    if (plan->max_units < c->kvp) return HELIX_ERR_CAPACITY;
     plan->grid = (sms / 2) * 2;  // clusters of two CTAs
     if (plan->grid < 2) return HELIX_ERR_UNSUPPORTED;
     plan->ticket_bytes = (((size_t)plan->units * 2 * sizeof(int32_t)) + 255) & ~size_t(255);
@@ -148,6 +155,7 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
   const size_t smem = nvfp4 ? gqa_nvfp4_smem_bytes(plan->units)
                             : gqa_partial_smem_bytes(c->head_dim, plan->units);
   if (smem > (size_t)max_smem) return HELIX_ERR_CAPACITY;
+  plan->max_units = plan->units;
   plan->grid = sms;
   plan->ticket_bytes = (((size_t)plan->units * sizeof(int32_t)) + 255) & ~size_t(255);
   plan->gticket_bytes =
@@ -319,8 +327,6 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
     m.kvp = c->kvp;
     m.max_pages = c->max_pages_per_shard;
     m.num_pages = c->num_pages;
-    m.units = units;
-    m.u0 = u0;
     m.scale_log2 = softmax_scale * 1.4426950408889634f;
     // latent pool as [pages * 64 rows][576], boxes of 64 columns x 64 rows; q as [B * 128][576],
     // boxes of 64 columns x 128 rows; 128-byte swizzle for the tensor-core operand layout
@@ -330,7 +336,16 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
         !encode_rows_map(&tmQ, const_cast<void*>(q), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
                          (uint64_t)c->batch * 128, 64, 128))
       return HELIX_ERR_CUDA;
-    return mla_partial_launch(tmC, tmQ, m, plan.grid, stream);
+    // request ranges of at most plan.max_units units each, one after another on the stream
+    // (they share the workspace; the unit tickets are back at zero after each launch)
+    const int per = plan.max_units / units_per_request;
+    for (int b = b_begin; b < b_end; b += per) {
+      m.u0 = b * units_per_request;
+      m.units = (min(b_end, b + per) - b) * units_per_request;
+      st = mla_partial_launch(tmC, tmQ, m, plan.grid, stream);
+      if (st != HELIX_OK) return st;
+    }
+    return HELIX_OK;
   }
 
   GqaParams p{};

@@ -158,3 +158,19 @@ def test_mla_many_short_units():
         res = _run(cache, w, q)
         assert cache.err_bits() == 0
         _check(w, q, lens, res, f"many units x{sharp}", heads=list(range(0, 128, 9)))
+
+
+def test_mla_batch_beyond_one_launch():
+    """240 requests x 8 shards = 1,920 (request, shard) units, more than one launch keeps in shared
+    memory: the partial runs as consecutive launches over request ranges, with the same results."""
+    rng = np.random.default_rng(11)
+    lens = [int(x) for x in rng.integers(1, 131, size=240)]
+    w = MLA.with_(B=240, S=max(lens), kvp=8)
+    cache = _gpu.make_cache(w)
+    _gpu.fill(cache, w, lens)
+    assert cache.err_bits() == 0
+    q = wl.query(w, "cuda")
+    res = _run(cache, w, q)
+    assert cache.err_bits() == 0
+    assert np.isfinite(res[2]).all() and np.isfinite(res[3]).all()
+    _check(w, q, lens, res, "1920 units", heads=[0, 63, 127])
