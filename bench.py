@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -109,7 +110,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.proc = None
         self.gpu = gpu_index
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # the raw samples go to a scratch file (HELIX_CLOCKS_DIR, else the system temp directory)
+        out_dir = os.environ.get("HELIX_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"helix_clocks_rank{gpu_index}.csv")
 
     def start(self):
         try:
