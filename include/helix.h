@@ -186,6 +186,27 @@ helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads,
                                 int32_t o_dtype, float* lse_out, helix_stream_t stream);
 
 /*
+ * The same combine over partials held in separate buffers, one per source shard, for the heads
+ * [head_begin, head_end) of every request. This is the owner's side of the exchange between GPUs
+ * (paper summary: after attention, an all-to-all takes the partial outputs and LSEs of every KV
+ * shard to the rank that owns a head group): on a multi-GPU node o_parts[s] / lses[s] are the
+ * source ranks' own buffers mapped into this process (CUDA IPC), read with plain loads over NVLink,
+ * so the exchange and the merge are one kernel.
+ *   o_parts[s]  fp32 [batch][num_q_heads][v_dim], lses[s] fp32 [batch][num_q_heads], s < nsrc
+ *               (host arrays of device-accessible pointers; 16-byte / 4-byte aligned)
+ *   o_out       [batch][head_end - head_begin][v_dim], bf16 (o_dtype 0) or fp32 (o_dtype 1)
+ *   lse_out     fp32 [batch][head_end - head_begin], may be NULL
+ * 1 <= nsrc <= HELIX_MAX_SOURCES; v_dim a multiple of 4. The arithmetic is helix_attn_combine's, in
+ * the same order: the results are bit-identical to it for the same partials.
+ */
+#define HELIX_MAX_SOURCES 16
+helix_status helix_attn_combine_sources(int32_t nsrc, const float* const* o_parts,
+                                        const float* const* lses, int32_t batch,
+                                        int32_t num_q_heads, int32_t v_dim, int32_t head_begin,
+                                        int32_t head_end, void* o_out, int32_t o_dtype,
+                                        float* lse_out, helix_stream_t stream);
+
+/*
  * helix_attn_partial followed by helix_attn_combine, in ONE launch for GQA caches: the CTA that
  * finishes the last of the kvp shards of a (request, KV head) group merges that group's rows into
  * o_out / lse_out in the same kernel (the same arithmetic as helix_attn_combine, bit for bit).

@@ -72,6 +72,8 @@ def _load():
     lib.helix_attn_partial_range.restype = I32
     lib.helix_attn_combine_range.argtypes = [I32, I32, I32, I32, I32, I32, P, P, P, I32, P, P]
     lib.helix_attn_combine_range.restype = I32
+    lib.helix_attn_combine_sources.argtypes = [I32, P, P, I32, I32, I32, I32, I32, P, I32, P, P]
+    lib.helix_attn_combine_sources.restype = I32
     lib.helix_attn_overlapped.argtypes = [cache_p, P, I32, F32, I32, P, P, P, I32, P, P, SZ, P, P,
                                           ctypes.POINTER(P)]
     lib.helix_attn_overlapped.restype = I32
@@ -244,6 +246,41 @@ def combine(o_partial: torch.Tensor, lse: torch.Tensor, out=None, lse_out=None,
     o_dtype = 0 if out.dtype == torch.bfloat16 else 1
     _check(lib.helix_attn_combine(P, B, Hq, dv, _ptr(o_partial), _ptr(lse), _ptr(out), o_dtype,
                                   _ptr(lse_out), _stream(stream)), "helix_attn_combine")
+    return out, lse_out
+
+
+MAX_SOURCES = 16
+
+
+def combine_sources(o_parts, lses, head_begin: int, head_end: int, out=None, lse_out=None,
+                    out_dtype=torch.bfloat16, want_lse=True, stream=None, ptrs=None):
+    """``helix_attn_combine_sources``: the combine over separate per-shard buffers (O [B][Hq][dv]
+    and lse [B][Hq] each) for the heads [head_begin, head_end). ``ptrs`` may give the sources as
+    raw device addresses instead (``[(o_addr, lse_addr), ...]``, e.g. other processes' buffers mapped
+    into this one); the shapes are then taken from ``o_parts[0]`` / ``lses[0]``. Returns (O, LSE or
+    None) with O [B][head_end - head_begin][dv]."""
+    B, Hq, dv = o_parts[0].shape
+    n = len(ptrs) if ptrs is not None else len(o_parts)
+    if ptrs is None:
+        if len(lses) != n:
+            raise ValueError("one lse buffer per O buffer")
+        for o, l in zip(o_parts, lses):
+            if tuple(o.shape) != (B, Hq, dv) or tuple(l.shape) != (B, Hq) or not (
+                    o.is_contiguous() and l.is_contiguous()):
+                raise ValueError("every source is a contiguous O [B][Hq][dv] and lse [B][Hq]")
+        ptrs = [(o.data_ptr(), l.data_ptr()) for o, l in zip(o_parts, lses)]
+    nh = head_end - head_begin
+    dev = o_parts[0].device
+    if out is None:
+        out = torch.empty(B, nh, dv, dtype=out_dtype, device=dev)
+    if lse_out is None and want_lse:
+        lse_out = torch.empty(B, nh, dtype=torch.float32, device=dev)
+    o_arr = (ctypes.c_void_p * n)(*[o for o, _ in ptrs])
+    l_arr = (ctypes.c_void_p * n)(*[l for _, l in ptrs])
+    o_dtype = 0 if out.dtype == torch.bfloat16 else 1
+    _check(lib.helix_attn_combine_sources(n, o_arr, l_arr, B, Hq, dv, head_begin, head_end,
+                                          _ptr(out), o_dtype, _ptr(lse_out), _stream(stream)),
+           "helix_attn_combine_sources")
     return out, lse_out
 
 

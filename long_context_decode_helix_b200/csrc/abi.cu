@@ -459,6 +459,33 @@ helix_status helix_attn_combine(int32_t kvp, int32_t batch, int32_t num_q_heads,
                                   o_dtype, lse_out, stream);
 }
 
+helix_status helix_attn_combine_sources(int32_t nsrc, const float* const* o_parts,
+                                        const float* const* lses, int32_t batch,
+                                        int32_t num_q_heads, int32_t v_dim, int32_t head_begin,
+                                        int32_t head_end, void* o_out, int32_t o_dtype,
+                                        float* lse_out, helix_stream_t stream) {
+  if (nsrc < 1 || nsrc > HELIX_MAX_SOURCES || o_parts == nullptr || lses == nullptr)
+    return HELIX_ERR_INVALID_ARG;
+  if (batch < 1 || num_q_heads < 1 || v_dim < 4 || v_dim % 4 != 0 || head_begin < 0 ||
+      head_end <= head_begin || head_end > num_q_heads)
+    return HELIX_ERR_INVALID_ARG;
+  if (o_out == nullptr || (o_dtype != 0 && o_dtype != 1) || !aligned16(o_out) ||
+      !aligned4(lse_out))
+    return HELIX_ERR_INVALID_ARG;
+  if ((int64_t)batch * num_q_heads * v_dim > INT32_MAX) return HELIX_ERR_CAPACITY;
+  CombineSources src{};
+  src.n = nsrc;
+  for (int s = 0; s < nsrc; ++s) {
+    if (o_parts[s] == nullptr || lses[s] == nullptr || !aligned16(o_parts[s]) ||
+        !aligned4(lses[s]))
+      return HELIX_ERR_INVALID_ARG;
+    src.o[s] = o_parts[s];
+    src.lse[s] = lses[s];
+  }
+  return combine_sources_launch(src, batch, num_q_heads, head_begin, head_end - head_begin, v_dim,
+                                o_out, o_dtype, lse_out, static_cast<cudaStream_t>(stream));
+}
+
 helix_status helix_attn_overlapped(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
                                    float softmax_scale, int32_t n_groups, float* o_partial,
                                    float* lse, void* o_out, int32_t o_dtype, float* lse_out,

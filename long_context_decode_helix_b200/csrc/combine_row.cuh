@@ -19,24 +19,26 @@
 
 namespace helix {
 
-// rows = B * Hq (the shard stride of o_part / lse); row = b * Hq + h; lanes stride v_dim by float4
-template <bool BF16_OUT>
-__device__ __forceinline__ void combine_row(int kvp, int rows, int row, int v_dim,
-                                            const float* o_part, const float* lse, void* o_out,
-                                            float* lse_out, int lane) {
+// The merge of one row over nsrc sources: lse_at(s) is source s's lse of the row, orow_at(s) its O
+// row (v_dim floats); lanes stride v_dim by float4. Every caller goes through this one function,
+// so the combine kernel, the fused combine and the combine over separate source buffers give
+// bit-identical results for the same partials.
+template <bool BF16_OUT, class LseAt, class ORowAt>
+__device__ __forceinline__ void combine_row_sources(int nsrc, int v_dim, LseAt lse_at,
+                                                    ORowAt orow_at, void* o_out_row,
+                                                    float* lse_out_elem, int lane) {
   float M = -INFINITY;
-  for (int s = 0; s < kvp; ++s) M = fmaxf(M, __ldcg(lse + (size_t)s * rows + row));
+  for (int s = 0; s < nsrc; ++s) M = fmaxf(M, lse_at(s));
   const float Mu = M == -INFINITY ? 0.f : M;
   float den = 0.f;
-  for (int s = 0; s < kvp; ++s) den += expf(__ldcg(lse + (size_t)s * rows + row) - Mu);
+  for (int s = 0; s < nsrc; ++s) den += expf(lse_at(s) - Mu);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   for (int c = lane * 4; c < v_dim; c += 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < kvp; ++s) {
-      const float w = expf(__ldcg(lse + (size_t)s * rows + row) - Mu);
+    for (int s = 0; s < nsrc; ++s) {
+      const float w = expf(lse_at(s) - Mu);
       if (w == 0.f) continue;  // empty shard: its O_s is never read
-      const float4 v =
-          __ldcg(reinterpret_cast<const float4*>(o_part + ((size_t)s * rows + row) * v_dim + c));
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(orow_at(s) + c));
       acc.x += w * v.x;
       acc.y += w * v.y;
       acc.z += w * v.z;
@@ -47,16 +49,32 @@ __device__ __forceinline__ void combine_row(int kvp, int rows, int row, int v_di
     acc.z *= inv;
     acc.w *= inv;
     if (BF16_OUT) {
-      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(o_out) + (size_t)row * v_dim + c;
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(o_out_row) + c;
       uint2 packed;
       packed.x = pack_bf16x2(acc.x, acc.y);
       packed.y = pack_bf16x2(acc.z, acc.w);
       *reinterpret_cast<uint2*>(o) = packed;
     } else {
-      *reinterpret_cast<float4*>(reinterpret_cast<float*>(o_out) + (size_t)row * v_dim + c) = acc;
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(o_out_row) + c) = acc;
     }
   }
-  if (lse_out != nullptr && lane == 0) lse_out[row] = den > 0.f ? Mu + logf(den) : -INFINITY;
+  if (lse_out_elem != nullptr && lane == 0) *lse_out_elem = den > 0.f ? Mu + logf(den) : -INFINITY;
+}
+
+// rows = B * Hq (the shard stride of o_part / lse); row = b * Hq + h; the kvp shards are one
+// contiguous [kvp][rows] (lse) and [kvp][rows][v_dim] (O) array
+template <bool BF16_OUT>
+__device__ __forceinline__ void combine_row(int kvp, int rows, int row, int v_dim,
+                                            const float* o_part, const float* lse, void* o_out,
+                                            float* lse_out, int lane) {
+  void* o_row = BF16_OUT ? static_cast<void*>(reinterpret_cast<__nv_bfloat16*>(o_out) +
+                                              (size_t)row * v_dim)
+                         : static_cast<void*>(reinterpret_cast<float*>(o_out) +
+                                              (size_t)row * v_dim);
+  combine_row_sources<BF16_OUT>(
+      kvp, v_dim, [&](int s) { return __ldcg(lse + (size_t)s * rows + row); },
+      [&](int s) { return o_part + ((size_t)s * rows + row) * v_dim; }, o_row,
+      lse_out != nullptr ? lse_out + row : nullptr, lane);
 }
 
 // Fused combine of the GQA partial kernels: called by every thread that `sync` covers after the

@@ -84,6 +84,16 @@ helix_status append_launch(const AppendParams& p, cudaStream_t stream);
 cudaError_t allow_max_dynamic_smem(const void* func);
 
 // rows = B * Hq (the shard stride of o_partial / lse); combines rows [row0, row0 + nrows)
+// Sources of a combine over separate buffers: source s holds O [B][Hq][v_dim] at o[s] and lse
+// [B][Hq] at lse[s] (device-accessible; on a multi-GPU node, peer mappings of other GPUs' buffers).
+struct CombineSources {
+  int n;
+  const float* o[HELIX_MAX_SOURCES];
+  const float* lse[HELIX_MAX_SOURCES];
+};
+helix_status combine_sources_launch(const CombineSources& src, int B, int Hq, int h0, int nh,
+                                    int v_dim, void* o_out, int o_dtype, float* lse_out,
+                                    cudaStream_t stream);
 helix_status combine_launch(int kvp, int rows, int row0, int nrows, int v_dim,
                             const float* o_partial, const float* lse, void* o_out, int o_dtype,
                             float* lse_out, cudaStream_t stream);
