@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="helix", choices=["helix", "reference"])
     ap.add_argument("--workload", default="gqa_s1m", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the steps launched from CUDA graphs (reported under 'graph')")
     ap.add_argument("--hopb-groups", type=int, default=4,
                     help="request groups of the two-stream HOP-B analogue, timed after the main "
                          "steps and reported under 'hopb' (0 = skip)")
@@ -309,7 +311,8 @@ def run_helix(args):
     lens = wl.seq_lens(w)
     dev = torch.device("cuda", local)
     K, W = args.steps, args.warmup
-    n_steps = K + W + (K if not args.no_e2e else 0) + (W + K if args.hopb_groups > 0 else 0)
+    n_steps = (K + W + (K if not args.no_e2e else 0) + (W + K if args.graph else 0) +
+               (W + K if args.hopb_groups > 0 else 0))
     S_cap = max(lens) + n_steps + 16
     if w.layout == "contig":  # size the contiguous shards for the history plus the new tokens
         w = w.with_(S_final=S_cap)
@@ -425,6 +428,36 @@ def run_helix(args):
         e2e = {"value": e2e_ms * 1e3, "unit": "us/step", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 
+    # --- optional: the same steps launched from CUDA graphs (one graph per step, captured outside
+    # the timed region), the form a caller uses when the step is launch-bound (short contexts) ---
+    graph = None
+    if args.graph:
+        graphs = []
+        cap_stream = torch.cuda.Stream(dev)
+        for i in range(K):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                one_step(si + i)
+            graphs.append(g)
+        torch.cuda.synchronize()
+        for g in graphs[:min(W, K)]:  # warm-up replays
+            g.replay()
+        barrier(world)
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for g in graphs:
+            g.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        graph_ms = max_over_ranks(g0.elapsed_time(g1) / K, world)
+        si += K
+        graph = {"us_per_step": graph_ms * 1e3, "steps": K,
+                 "how": "each step captured once in a CUDA graph, then replayed back to back"}
+        del graphs
+        assert cache.err_bits() == 0, "a graph-launched step reported a device error"
+
     # --- HOP-B analogue: the combine of request group g on a second stream overlaps the partial of
     # group g+1; same append, same inputs, timed like the main steps ---
     hopb = None
@@ -504,6 +537,7 @@ def run_helix(args):
             "e2e": e2e,
             "clocks": clk,
             "hopb": hopb,
+            "graph": graph,
             "read_probe": read_probe,
         }
         if not args.no_cpu_baseline and world == 1:
