@@ -50,6 +50,25 @@ def test_combine_rejects_bad_arguments(hx):
     assert f(1, 1, 1, 4, ctypes.c_void_p(8), buf, buf, 0, None, None) == 1  # misaligned
 
 
+def test_combine_sources_rejects_bad_arguments(hx):
+    f = hx.lib.helix_attn_combine_sources
+    buf = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+
+    def arr(*p):
+        return (ctypes.c_void_p * len(p))(*p)
+
+    o1, l1 = arr(16), arr(16)
+    assert f(0, o1, l1, 1, 4, 8, 0, 4, buf, 0, None, None) == 1  # no source
+    assert f(17, arr(*([16] * 17)), arr(*([16] * 17)), 1, 4, 8, 0, 4, buf, 0, None, None) == 1
+    assert f(1, o1, l1, 1, 4, 8, 2, 2, buf, 0, None, None) == 1  # empty head range
+    assert f(1, o1, l1, 1, 4, 8, 0, 5, buf, 0, None, None) == 1  # past the last head
+    assert f(1, o1, l1, 1, 4, 6, 0, 4, buf, 0, None, None) == 1  # v_dim not a multiple of 4
+    assert f(1, arr(8), l1, 1, 4, 8, 0, 4, buf, 0, None, None) == 1  # misaligned source O
+    assert f(1, arr(None), l1, 1, 4, 8, 0, 4, buf, 0, None, None) == 1  # null source
+    assert f(1, o1, l1, 1, 4, 8, 0, 4, buf, 3, None, None) == 1  # bad o_dtype
+    assert f(1, None, l1, 1, 4, 8, 0, 4, buf, 0, None, None) == 1  # no source array
+
+
 def _struct(hx, **kw):
     base = dict(kind=0, kv_dtype=0, layout=0, kvp=8, batch=8, num_kv_heads=8, head_dim=128,
                 v_dim=128, page_tokens=64, rr_block=16, contig_chunk=0, num_pages=16,
