@@ -319,11 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
         }
       }
     }
-    // ---- online softmax over the page (base 2, lazy reference maximum)
-#pragma unroll
-    for (int n = 0; n < 8; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[n][e] *= sl2;
+    // ---- online softmax over the page (base 2, lazy reference maximum). The logit scale (times
+    // log2 e, positive) is applied inside the exponent, fma(s, sl2, -m); the row maximum is taken
+    // over the raw scores and scaled once.
     if (nvalid < kPage) {
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
@@ -340,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
     }
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2)) * sl2;
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2)) * sl2;
     const bool up0 = mx0 > m_ref[0] + kLazy, up1 = mx1 > m_ref[1] + kLazy;
     if (__any_sync(0xffffffffu, up0 || up1)) {
       const float n0 = up0 ? mx0 : m_ref[0], n1 = up1 ? mx1 : m_ref[1];
@@ -367,10 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t pa[4];
-      pa[0] = pack_f16x2(fast_exp2(s[2 * cc][0] - mu0), fast_exp2(s[2 * cc][1] - mu0));
-      pa[1] = pack_f16x2(fast_exp2(s[2 * cc][2] - mu1), fast_exp2(s[2 * cc][3] - mu1));
-      pa[2] = pack_f16x2(fast_exp2(s[2 * cc + 1][0] - mu0), fast_exp2(s[2 * cc + 1][1] - mu0));
-      pa[3] = pack_f16x2(fast_exp2(s[2 * cc + 1][2] - mu1), fast_exp2(s[2 * cc + 1][3] - mu1));
+      pa[0] = pack_f16x2(fast_exp2(fmaf(s[2 * cc][0], sl2, -mu0)),
+                         fast_exp2(fmaf(s[2 * cc][1], sl2, -mu0)));
+      pa[1] = pack_f16x2(fast_exp2(fmaf(s[2 * cc][2], sl2, -mu1)),
+                         fast_exp2(fmaf(s[2 * cc][3], sl2, -mu1)));
+      pa[2] = pack_f16x2(fast_exp2(fmaf(s[2 * cc + 1][0], sl2, -mu0)),
+                         fast_exp2(fmaf(s[2 * cc + 1][1], sl2, -mu0)));
+      pa[3] = pack_f16x2(fast_exp2(fmaf(s[2 * cc + 1][2], sl2, -mu1)),
+                         fast_exp2(fmaf(s[2 * cc + 1][3], sl2, -mu1)));
       // token pairs (2t, 2t+1) and (2t+8, 2t+9) of the chunk; a pair row's 16-byte chunks are
       // stored XOR-swizzled by 2 (pair mod 4) = 2t, so a quarter-warp hits every bank once
       const int pa_ = 8 * cc + t4, pb_ = pa_ + 4;

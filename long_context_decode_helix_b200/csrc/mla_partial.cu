@@ -725,12 +725,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       keep_alive(sv);
       __syncwarp();
       if (lane == 0) remote_arrive_relaxed(xfree_peer);
-      if (nvalid == kTok && tile_ok) {
+      // the logit scale (times log2 e, positive) is applied inside the exponent below,
+      // fma(s, sl2, -m); the row maximum is taken over the raw scores and scaled once
+      if (nvalid < kTok || !tile_ok) {
 #pragma unroll
-        for (int c = 0; c < kTok; ++c) sv[c] *= sl2;
-      } else {
-#pragma unroll
-        for (int c = 0; c < kTok; ++c) sv[c] = (c < nvalid && tile_ok) ? sv[c] * sl2 : -INFINITY;
+        for (int c = 0; c < kTok; ++c) sv[c] = (c < nvalid && tile_ok) ? sv[c] : -INFINITY;
       }
       float mx;
       {  // tree reduction of the row maximum
@@ -741,7 +740,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) t[c] = fmaxf(t[c], t[c + 8]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) t[c] = fmaxf(t[c], t[c + 4]);
-        mx = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
+        mx = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3])) * sl2;
       }
       // V rows past the end of the history, or all of a tile whose page id is out of range (not
       // loaded: stale or never-written shared memory), are zeroed before the P V product reads
@@ -779,8 +778,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float ps[16];
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
-        const float p0 = fast_exp2(sv[c] - mb), p1 = fast_exp2(sv[c + 1] - mb);
-        const float p2 = fast_exp2(sv[c + 32] - mb), p3 = fast_exp2(sv[c + 33] - mb);
+        const float p0 = fast_exp2(fmaf(sv[c], sl2, -mb)), p1 = fast_exp2(fmaf(sv[c + 1], sl2, -mb));
+        const float p2 = fast_exp2(fmaf(sv[c + 32], sl2, -mb));
+        const float p3 = fast_exp2(fmaf(sv[c + 33], sl2, -mb));
         ps[c / 2] = (p0 + p1) + (p2 + p3);
         pk[c / 2] = pack_bf16x2(p0, p1);
         pk[16 + c / 2] = pack_bf16x2(p2, p3);
