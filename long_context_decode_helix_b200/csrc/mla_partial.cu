@@ -37,14 +37,15 @@
 // so two tiles are in the softmax at once; thread h of a group owns head h = TMEM lane h), 8 TMA
 // producer (and L2 prefetch one tile ahead), 9 score-MMA issuer and TMEM allocator, 10 P V issuer
 // (one thread each, so a ready P V never waits behind a score tile). Each group has its own TMEM
-// score buffer, so the tensor
-// core computes the next tile's scores while a group works on its tile. The groups share one reference maximum per head, handed from the owner
-// of tile i-1 to the owner of tile i through shared memory and a named barrier; each group keeps its
-// own running sum, and the two are merged at the end of a segment. O is rescaled lazily: the exponent base only moves when
-// a row maximum grows by more than 8 (in base-2 units), so weights stay below 2^8 and the 256-column
-// TMEM rescale is rare. Work is split over the (request, shard) units exactly as in the GQA kernel:
-// each cluster takes an equal contiguous range of 64-token tiles; split units are merged by the last
-// arriving cluster, per value half.
+// score buffer, so the tensor core computes the next tile's scores while a group works on its
+// tile. The groups share one reference maximum per head, handed from the owner of tile i-1 to the
+// owner of tile i through shared memory and an mbarrier per 32-row slice; each group keeps its own
+// running sum, and the two are merged at the end of a segment. O is rescaled lazily: the exponent
+// base only moves when a row maximum grows by more than 8 (in base-2 units), so weights stay below
+// 2^8 and the 256-column TMEM rescale is rare. The logit scale is applied inside the exponent.
+// Work is split over the (request, shard) units exactly as in the GQA kernel: each cluster takes an
+// equal contiguous range of 64-token tiles; split units are merged by the last arriving cluster,
+// per value half.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
