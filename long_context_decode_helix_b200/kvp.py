@@ -117,20 +117,25 @@ class KVPExchange:
             torch.cuda.current_stream(self.device).synchronize()
         dist.barrier(group=self.group)
 
+    def _merge(self, o_parts, lses, out, lse_out, out_dtype):
+        if self.h1 == self.h0:  # more ranks than heads: this rank owns none
+            return (torch.empty(self.B, 0, self.dv, dtype=out_dtype, device=self.device),
+                    torch.empty(self.B, 0, dtype=torch.float32, device=self.device))
+        return self._combine(o_parts, lses, self.h0, self.h1, out=out, lse_out=lse_out,
+                             out_dtype=out_dtype)
+
     def combine(self, out=None, lse_out=None, out_dtype=torch.bfloat16):
         """Exchange the partials and merge the owned heads; returns (O, LSE)."""
         if self.mode == "peer":
             self._sync()  # every rank's partial is written
             o_parts = [o[0] for o, _ in self._peers]
             lses = [l[0] for _, l in self._peers]
-            res = self._combine(o_parts, lses, self.h0, self.h1, out=out, lse_out=lse_out,
-                                out_dtype=out_dtype)
+            res = self._merge(o_parts, lses, out, lse_out, out_dtype)
             self._sync()  # nobody reads a partial any more: it may be overwritten
             return res
         dist.all_gather_into_tensor(self._all_o, self.o_partial, group=self.group)
         dist.all_gather_into_tensor(self._all_lse, self.lse, group=self.group)
-        return self._combine(list(self._all_o), list(self._all_lse), self.h0, self.h1, out=out,
-                             lse_out=lse_out, out_dtype=out_dtype)
+        return self._merge(list(self._all_o), list(self._all_lse), out, lse_out, out_dtype)
 
     def close(self):
         """Drop the mappings of the other ranks' buffers (every rank calls it)."""

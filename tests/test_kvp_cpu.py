@@ -77,23 +77,24 @@ def _rank_main(rank, world, port, q, K, V, lens, scale, errors):
         for _ in range(2):  # twice: the exchange is reusable step after step
             O, L = ex.combine()
         h0, h1 = kvp.owned_heads(rank, world, Hq)
-        assert tuple(O.shape) == (B, h1 - h0, dv)
+        assert tuple(O.shape) == (B, h1 - h0, dv) and tuple(L.shape) == (B, h1 - h0)
         # the partials travel in fp32 (the kernels' buffers): agreement to fp32 rounding
         for b in range(B):
             Oref, Lref = oracle.attend(q[b, h0:h1], K[b, : lens[b]], V[b, : lens[b]], scale)
-            np.testing.assert_allclose(O[b].numpy(), Oref, rtol=1e-5, atol=1e-6)
-            np.testing.assert_allclose(L[b].numpy(), Lref, rtol=1e-6, atol=1e-6)
+            np.testing.assert_allclose(O[b].double().numpy(), Oref, rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(L[b].double().numpy(), Lref, rtol=1e-6, atol=1e-6)
         ex.close()
         dist.destroy_process_group()
     except Exception as e:  # reported to the parent, which fails the test
         errors.put(f"rank {rank}: {type(e).__name__}: {e}")
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_gather_exchange_equals_unsharded_attention(world):
-    """Every rank ends with exactly the unsharded attention of the heads it owns."""
+@pytest.mark.parametrize("world,Hq", [(2, 6), (3, 6), (3, 2)])
+def test_gather_exchange_equals_unsharded_attention(world, Hq):
+    """Every rank ends with the unsharded attention of the heads it owns (none, when there are
+    more ranks than heads), to the fp32 rounding of the exchanged partials."""
     rng = np.random.default_rng(5)
-    B, Hq, d, dv = 2, 6, 16, 8
+    B, d, dv = 2, 16, 8
     lens = [70, 3]  # the second request has no token on some ranks: empty partials
     S = max(lens)
     q = rng.standard_normal((B, Hq, d))
