@@ -34,6 +34,22 @@ def test_every_declared_symbol_is_exported(hx):
         assert hasattr(hx.lib, n), f"libhelix.so does not export {n}"
 
 
+def test_header_is_plain_c():
+    """include/helix.h compiles as C (no C++ in the ABI) and as C++."""
+    import shutil
+    import subprocess
+
+    inc = os.path.join(ROOT, "include")
+    for cc, lang in (("gcc", "c"), ("g++", "c++")):
+        exe = shutil.which(cc)
+        if exe is None:
+            pytest.skip(f"{cc} not found")
+        r = subprocess.run([exe, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang, "-I",
+                            "/usr/local/cuda/include", os.path.join(inc, "helix.h")],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
 def test_status_strings(hx):
     for code, name in hx.STATUS_NAMES.items():
         assert hx.lib.helix_status_string(code).decode() == name
