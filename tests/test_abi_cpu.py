@@ -44,9 +44,9 @@ def test_header_is_plain_c():
         exe = shutil.which(cc)
         if exe is None:
             pytest.skip(f"{cc} not found")
-        r = subprocess.run([exe, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang, "-I",
-                            "/usr/local/cuda/include", os.path.join(inc, "helix.h")],
-                           capture_output=True, text=True)
+        # no CUDA header is needed: the ABI uses only standard C types and opaque handles
+        r = subprocess.run([exe, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang,
+                            os.path.join(inc, "helix.h")], capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
 
 
