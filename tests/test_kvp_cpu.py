@@ -35,6 +35,24 @@ def test_append_valid_marks_the_owner_of_each_new_token():
     assert sum(kvp.append_valid(pos, r, world) for r in range(world)).tolist() == [1] * len(pos)
 
 
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_decode_loop_appends_build_each_ranks_shard(world):
+    """Token by token, each rank appends exactly the new tokens ``append_valid`` gives it; after S
+    steps its history is its shard of the layout, for requests of different lengths."""
+    lens0, S = [0, 37], 300
+    held = [[[] for _ in lens0] for _ in range(world)]
+    for step in range(S):
+        pos = [L + step for L in lens0]
+        for r in range(world):
+            for b, v in enumerate(kvp.append_valid(pos, r, world).tolist()):
+                if v:
+                    held[r][b].append(pos[b])
+    for r in range(world):
+        for b, L0 in enumerate(lens0):
+            want = [t for t in kvp.local_positions(L0 + S, r, world).tolist() if t >= L0]
+            assert held[r][b] == want
+
+
 @pytest.mark.parametrize("world,Hq", [(1, 128), (2, 128), (3, 128), (8, 128), (4, 6), (16, 16)])
 def test_owned_heads_partition_the_heads(world, Hq):
     ranges = [kvp.owned_heads(r, world, Hq) for r in range(world)]
