@@ -48,7 +48,7 @@ typedef enum {
   HELIX_ERR_UNSUPPORTED = 2, /* a shape/dtype combination no kernel is built for */
   HELIX_ERR_CAPACITY = 3,    /* the call cannot fit its work in the sizes given */
   HELIX_ERR_CUDA = 4,        /* a CUDA runtime error (launch failure, no device, ...) */
-  HELIX_ERR_TIMEOUT = 5      /* reserved for host-side waits with a limit */
+  HELIX_ERR_TIMEOUT = 5      /* a host-side wait with a limit ran out (helix_stream_wait) */
 } helix_status;
 
 /* Bits written (OR-ed) into *err_word by the kernels. */
@@ -296,8 +296,11 @@ helix_status helix_decode_overlapped(const helix_kv_cache* cache, const void* q,
  * call cudaMalloc. The call allocates nothing.
  *   - Returns HELIX_ERR_CAPACITY, launching nothing, when this cache shape needs more scratch than
  *     HELIX_NOALLOC_SCRATCH_BYTES (see helix_attn_workspace_size).
+ *   - Every argument is checked before anything is enqueued: a rejected call launches nothing and
+ *     does not touch the shared array.
  *   - The first call on each device looks up the array's device address (once, with that device
- *     current); make that first call before any stream capture.
+ *     current); make that first call before any stream capture. The address is kept for the life
+ *     of the process: after cudaDeviceReset on a device, do not call this entry point there again.
  *   - Each call zeroes the scratch it uses (an async memset on `stream`) before the kernel runs.
  *   - All calls on one device share the array: calls that may run concurrently on the GPU race and
  *     must be ordered by the caller (one stream, or events).
@@ -306,6 +309,21 @@ helix_status helix_decode_overlapped(const helix_kv_cache* cache, const void* q,
 helix_status helix_attn_partial_noalloc(const helix_kv_cache* cache, const void* q,
                                         int32_t num_q_heads, float softmax_scale,
                                         float* o_partial, float* lse, helix_stream_t stream);
+
+/*
+ * Wait, with a wall-clock limit, for the work enqueued on `stream` so far. The library has no
+ * counterpart in the pages; this is the host side of its failure handling: where
+ * cudaStreamSynchronize would block for as long as the GPU takes, this call records `event` on
+ * `stream` and polls it (cudaEventQuery) until the work is done or `limit_us` microseconds have
+ * passed.
+ *   event    a CUDA event created by the caller (timing disabled is best); re-recorded here.
+ *   limit_us the limit in microseconds (0 polls once).
+ * Returns HELIX_OK when all of the stream's earlier work has finished, HELIX_ERR_TIMEOUT when the
+ * limit passed first (the work is still enqueued and may finish later: the caller decides whether
+ * to wait again or give up), HELIX_ERR_CUDA when recording or querying the event fails (including
+ * an error raised by the stream's earlier work), HELIX_ERR_INVALID_ARG for a NULL event.
+ */
+helix_status helix_stream_wait(helix_stream_t stream, helix_event_t event, uint64_t limit_us);
 
 /* Static, human-readable name of a status code. */
 const char* helix_status_string(helix_status status);

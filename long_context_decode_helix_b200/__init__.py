@@ -80,6 +80,8 @@ def _load():
     lib.helix_decode_overlapped.argtypes = [cache_p, P, I32, F32, I32, P, P, P, P, I32, P, P, P, P,
                                             I32, P, P, SZ, P, P, ctypes.POINTER(P)]
     lib.helix_decode_overlapped.restype = I32
+    lib.helix_stream_wait.argtypes = [P, P, ctypes.c_uint64]
+    lib.helix_stream_wait.restype = I32
     lib.helix_status_string.argtypes = [I32]
     lib.helix_status_string.restype = ctypes.c_char_p
     lib.helix_version.argtypes = []
@@ -425,6 +427,24 @@ def decode_overlapped(cache: KVCache, q: torch.Tensor, softmax_scale: float, ove
                                        _stream(stream), _stream(overlap.stream_b),
                                        overlap._handles), "helix_decode_overlapped")
     return out, lse_out
+
+
+HELIX_ERR_TIMEOUT = 5
+_wait_events = {}
+
+
+def wait(stream=None, limit_s: float = 60.0):
+    """Wait for the work enqueued on ``stream`` (default: the current stream) with a wall-clock
+    limit (``helix_stream_wait``). Raises ``HelixError`` with status HELIX_ERR_TIMEOUT when the limit
+    passes first (the work stays enqueued), HELIX_ERR_CUDA when the stream's work failed."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    ev = _wait_events.get(s.device)
+    if ev is None:
+        ev = torch.cuda.Event()
+        ev.record(s)  # torch creates the CUDA event lazily, on its first record
+        _wait_events[s.device] = ev
+    _check(lib.helix_stream_wait(_stream(s), ctypes.c_void_p(ev.cuda_event),
+                                 int(max(0.0, limit_s) * 1e6)), "helix_stream_wait")
 
 
 def decode_step(cache: KVCache, q, k_new, v_new=None, softmax_scale=None, k_scale=None,

@@ -8,6 +8,7 @@
 
 #include <mutex>
 
+#include "bounded_wait.h"
 #include "helix.h"
 #include "internal.h"
 
@@ -288,24 +289,34 @@ namespace {
 
 // The partial attention of requests [b_begin, b_end); with o_out non-null (GQA only) the kernel
 // also merges the shards of every KV-head group into o_out / lse_out (fused combine).
-helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
-                          float softmax_scale, int32_t b_begin, int32_t b_end, float* o_partial,
-                          float* lse, void* workspace, size_t workspace_bytes, void* o_out,
-                          int32_t o_dtype, float* lse_out, cudaStream_t stream) {
+// Every check of a partial call except those on the workspace; fills the launch plan.
+helix_status check_partial(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                           float softmax_scale, int32_t b_begin, int32_t b_end,
+                           const float* o_partial, const float* lse, const void* o_out,
+                           int32_t o_dtype, const float* lse_out, PartialPlan* plan) {
   if (c == nullptr || b_begin < 0 || b_end < b_begin || b_end > c->batch)
     return HELIX_ERR_INVALID_ARG;
-  PartialPlan plan;
-  helix_status st = plan_partial(c, num_q_heads, &plan);
+  helix_status st = plan_partial(c, num_q_heads, plan);
   if (st != HELIX_OK) return st;
-  if (q == nullptr || o_partial == nullptr || lse == nullptr || workspace == nullptr)
-    return HELIX_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(o_partial) || !aligned4(lse) || !aligned16(workspace))
-    return HELIX_ERR_INVALID_ARG;
-  if (workspace_bytes < plan.total()) return HELIX_ERR_INVALID_ARG;
+  if (q == nullptr || o_partial == nullptr || lse == nullptr) return HELIX_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o_partial) || !aligned4(lse)) return HELIX_ERR_INVALID_ARG;
   if (o_out != nullptr && (c->kind != HELIX_ATTN_GQA || (o_dtype != 0 && o_dtype != 1) ||
                            !aligned16(o_out) || !aligned4(lse_out)))
     return HELIX_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return HELIX_ERR_INVALID_ARG;
+  return HELIX_OK;
+}
+
+helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                          float softmax_scale, int32_t b_begin, int32_t b_end, float* o_partial,
+                          float* lse, void* workspace, size_t workspace_bytes, void* o_out,
+                          int32_t o_dtype, float* lse_out, cudaStream_t stream) {
+  PartialPlan plan;
+  helix_status st = check_partial(c, q, num_q_heads, softmax_scale, b_begin, b_end, o_partial,
+                                  lse, o_out, o_dtype, lse_out, &plan);
+  if (st != HELIX_OK) return st;
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < plan.total())
+    return HELIX_ERR_INVALID_ARG;
   if (b_end == b_begin) return HELIX_OK;
   // units are ordered request-major, so a request range is a contiguous unit range
   const int units_per_request = plan.units / c->batch;
@@ -393,9 +404,41 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
 }
 
 }  // namespace
+
+helix_status validate_partial_call(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                                   float softmax_scale, const float* o_partial, const float* lse,
+                                   size_t* workspace_bytes) {
+  PartialPlan plan;
+  helix_status st = check_partial(c, q, num_q_heads, softmax_scale, 0, c ? c->batch : 0,
+                                  o_partial, lse, nullptr, 0, nullptr, &plan);
+  if (st != HELIX_OK) return st;
+  *workspace_bytes = plan.total();
+  return HELIX_OK;
+}
+
 }  // namespace helix
 
 extern "C" {
+
+helix_status helix_stream_wait(helix_stream_t stream, helix_event_t event, uint64_t limit_us) {
+  if (event == nullptr) return HELIX_ERR_INVALID_ARG;
+  auto ev = reinterpret_cast<cudaEvent_t>(event);
+  if (cudaEventRecord(ev, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return HELIX_ERR_CUDA;
+  return poll_with_limit(
+      [ev]() {
+        const cudaError_t e = cudaEventQuery(ev);
+        if (e == cudaSuccess) return PollResult::kDone;
+        if (e == cudaErrorNotReady) {
+          // a pending query is not an error: if the runtime recorded it as the last error, clear
+          // it so that a later launch check does not read it as a failure
+          if (cudaPeekAtLastError() == cudaErrorNotReady) (void)cudaGetLastError();
+          return PollResult::kPending;
+        }
+        return PollResult::kError;
+      },
+      limit_us);
+}
 
 helix_status helix_attn_partial_range(const helix_kv_cache* c, const void* q,
                                       int32_t num_q_heads, float softmax_scale, int32_t b_begin,

@@ -80,6 +80,12 @@ struct AppendParams {
 };
 helix_status append_launch(const AppendParams& p, cudaStream_t stream);
 
+// Every host-side check of helix_attn_partial over the whole batch except those on the workspace
+// (launches nothing); on success *workspace_bytes is the scratch the call needs.
+helix_status validate_partial_call(const helix_kv_cache* c, const void* q, int32_t num_q_heads,
+                                   float softmax_scale, const float* o_partial, const float* lse,
+                                   size_t* workspace_bytes);
+
 // Raises a kernel's dynamic shared-memory limit to the device maximum, once per (kernel, device).
 cudaError_t allow_max_dynamic_smem(const void* func);
 

@@ -16,7 +16,9 @@
 // Host code cannot use the array's name as a device address: in host code it names a host-side
 // stand-in. The device address is looked up with cudaGetSymbolAddress once per device, with that
 // device current, on the first call made on it; that first call should therefore be made before
-// any stream capture begins.
+// any stream capture begins. The cached address belongs to the device's context as it was at that
+// first call: after cudaDeviceReset on a device this entry point must not be used there again in
+// the same process (the library's module, and with it the array, is reloaded at a new address).
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -24,6 +26,7 @@
 #include <mutex>
 
 #include "helix.h"
+#include "internal.h"
 
 static __device__ __align__(256) unsigned char helix_noalloc_scratch[HELIX_NOALLOC_SCRATCH_BYTES];
 
@@ -55,8 +58,11 @@ extern "C" helix_status helix_attn_partial_noalloc(const helix_kv_cache* cache, 
                                                    int32_t num_q_heads, float softmax_scale,
                                                    float* o_partial, float* lse,
                                                    helix_stream_t stream) {
+  // every argument is checked before anything is enqueued: a rejected call touches neither the
+  // stream nor the shared scratch (which an earlier call may still be using)
   size_t need = 0;
-  helix_status st = helix_attn_workspace_size(cache, num_q_heads, &need);
+  helix_status st = helix::validate_partial_call(cache, q, num_q_heads, softmax_scale, o_partial,
+                                                 lse, &need);
   if (st != HELIX_OK) return st;
   if (need > (size_t)HELIX_NOALLOC_SCRATCH_BYTES) return HELIX_ERR_CAPACITY;
   void* scratch = nullptr;

@@ -143,3 +143,53 @@ class KVPExchange:
         if self.device.type == "cuda":
             torch.cuda.synchronize(self.device)
         dist.barrier(group=self.group)
+
+
+class KVPDecodeRank:
+    """One rank's side of a KV-parallel decode step, as a decode loop runs it.
+
+    Per step: the new token of every request is appended on the rank that owns its history
+    position (``append_valid``), every rank runs the partial attention over its local shard for all
+    heads into the exchange's buffers, and ``exchange.combine()`` returns the LSE-combined output of
+    the heads this rank owns.
+
+    ``append_fn(rows, n_valid)`` appends one new row per request where ``n_valid[b]`` is 1 (for the
+    library: ``helix.append(cache, **rows, n_valid=n_valid)`` on the rank's kvp = 1 cache);
+    ``partial_fn(q, o_partial, lse)`` writes this rank's partials (``helix.partial``). Both are
+    arguments so the loop's host logic can be exercised without a GPU.
+    """
+
+    def __init__(self, exchange: KVPExchange, append_fn, partial_fn, lengths, rr_block: int = 16):
+        self.ex = exchange
+        self.append_fn = append_fn
+        self.partial_fn = partial_fn
+        self.rr_block = rr_block
+        self.lengths = [int(L) for L in lengths]  # every request's global history length
+
+    def owned_counts(self):
+        """How many tokens of each request's current history this rank stores."""
+        r, w, k = self.ex.rank, self.ex.world, self.rr_block
+        out = []
+        for L in self.lengths:
+            full, rem = divmod(L, k * w)  # whole rounds of the rotation, then a partial round
+            out.append(full * k + min(max(rem - r * k, 0), k))
+        return out
+
+    def append(self, rows):
+        """Append the step's new token of every request (on its owner only)."""
+        nv = append_valid(self.lengths, self.ex.rank, self.ex.world, self.rr_block,
+                          device=self.ex.device)
+        self.append_fn(rows, nv)
+        self.lengths = [L + 1 for L in self.lengths]
+
+    def attend(self, q, out=None, lse_out=None, out_dtype=torch.bfloat16):
+        """Partial attention over the local shard, then the exchange and combine."""
+        self.partial_fn(q, self.ex.o_partial, self.ex.lse)
+        return self.ex.combine(out=out, lse_out=lse_out, out_dtype=out_dtype)
+
+    def step(self, rows, q, out=None, lse_out=None, out_dtype=torch.bfloat16):
+        """One decode step: append, partial, exchange + combine; returns (O, LSE) of the owned
+        heads."""
+        self.append(rows)
+        return self.attend(q, out, lse_out, out_dtype)
+

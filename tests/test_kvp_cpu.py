@@ -135,3 +135,82 @@ def test_gather_exchange_equals_unsharded_attention(world, Hq):
         msgs.append(errors.get())
     assert not msgs, "\n".join(msgs)
     assert all(p.exitcode == 0 for p in procs)
+
+
+def _decode_rank_main(rank, world, port, q, K, V, lens0, steps, scale, errors):
+    """One rank of a KV-parallel decode loop (``kvp.KVPDecodeRank``, as ``bench.py --kvp-ranks``
+    drives it) with the oracle standing in for the append, partial and combine kernels."""
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        B, Hq, _ = q.shape
+        dv = V.shape[-1]
+        # the rank's local history: its tokens of every request's prefill
+        held = [[int(t) for t in kvp.local_positions(L, rank, world)] for L in lens0]
+
+        def append_fn(rows, n_valid):
+            for b, v in enumerate(n_valid.tolist()):
+                if v:
+                    held[b].append(rows["pos"][b])
+
+        def partial_fn(q_, o_part, lse):
+            for b in range(B):
+                idx = np.array(held[b], dtype=np.int64)
+                for h in range(Hq):
+                    if len(idx) == 0:  # an empty shard: O_s = 0, lse_s = -inf
+                        o_part[0, b, h] = 0.0
+                        lse[0, b, h] = float("-inf")
+                        continue
+                    o, l = oracle.attend(q_[b, h:h + 1], K[b, idx], V[b, idx], scale)
+                    o_part[0, b, h] = torch.from_numpy(o[0])
+                    lse[0, b, h] = float(l[0])
+
+        ex = kvp.KVPExchange(B, Hq, dv, "cpu", mode="gather", combine_fn=_oracle_combine)
+        dec = kvp.KVPDecodeRank(ex, append_fn, partial_fn, lens0)
+        assert dec.owned_counts() == [len(h) for h in held]
+        for s in range(steps):
+            pos = [L + s for L in lens0]
+            O, L = dec.step({"pos": pos}, q)
+        assert dec.owned_counts() == [len(h) for h in held]
+        h0, h1 = kvp.owned_heads(rank, world, Hq)
+        for b in range(B):
+            S = lens0[b] + steps
+            Oref, Lref = oracle.attend(q[b, h0:h1], K[b, :S], V[b, :S], scale)
+            np.testing.assert_allclose(O[b].double().numpy(), Oref, rtol=1e-5, atol=1e-6)
+            np.testing.assert_allclose(L[b].double().numpy(), Lref, rtol=1e-6, atol=1e-6)
+        ex.close()
+        dist.destroy_process_group()
+    except Exception as e:  # reported to the parent, which fails the test
+        errors.put(f"rank {rank}: {type(e).__name__}: {e}")
+
+
+@pytest.mark.parametrize("world", [2])
+def test_decode_loop_over_ranks_equals_unsharded_attention(world):
+    """Prefill, then 40 decode steps: every new token lands on exactly one rank, and after the last
+    step each rank's owned heads equal unsharded attention over the whole history."""
+    rng = np.random.default_rng(9)
+    B, Hq, d, dv, steps = 2, 4, 16, 8, 40
+    lens0 = [33, 5]
+    S = max(lens0) + steps
+    q = rng.standard_normal((B, Hq, d))
+    K = rng.standard_normal((B, S, d))
+    V = rng.standard_normal((B, S, dv))
+    ctx = mp.get_context("spawn")
+    errors = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_decode_rank_main,
+                         args=(r, world, port, q, K, V, lens0, steps, 0.25, errors))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    msgs = []
+    while not errors.empty():
+        msgs.append(errors.get())
+    assert not msgs, "\n".join(msgs)
+    assert all(p.exitcode == 0 for p in procs)
