@@ -52,6 +52,13 @@ def append_valid(positions, rank: int, world: int, rr_block: int = 16, device="c
                         dtype=torch.int32, device=device)
 
 
+def owned_count(L: int, rank: int, world: int, rr_block: int = 16) -> int:
+    """How many of the history positions t < L rank ``rank`` stores: whole rounds of the rotation
+    give rr_block tokens each, then the rank's part of the last, partial round."""
+    full, rem = divmod(int(L), rr_block * world)
+    return full * rr_block + min(max(rem - rank * rr_block, 0), rr_block)
+
+
 def local_positions(S: int, rank: int, world: int, rr_block: int = 16) -> torch.Tensor:
     """The history positions t < S that rank ``rank`` stores, in increasing order (its local
     history, as a kvp = 1 cache holds it)."""
@@ -168,12 +175,7 @@ class KVPDecodeRank:
 
     def owned_counts(self):
         """How many tokens of each request's current history this rank stores."""
-        r, w, k = self.ex.rank, self.ex.world, self.rr_block
-        out = []
-        for L in self.lengths:
-            full, rem = divmod(L, k * w)  # whole rounds of the rotation, then a partial round
-            out.append(full * k + min(max(rem - r * k, 0), k))
-        return out
+        return [owned_count(L, self.ex.rank, self.ex.world, self.rr_block) for L in self.lengths]
 
     def append(self, rows):
         """Append the step's new token of every request (on its owner only)."""
