@@ -305,7 +305,9 @@ helix_status helix_decode_overlapped(const helix_kv_cache* cache, const void* q,
  *   - All calls on one device share the array: calls that may run concurrently on the GPU race and
  *     must be ordered by the caller (one stream, or events).
  */
-#define HELIX_NOALLOC_SCRATCH_BYTES (4u << 20)
+/* 48 MiB: an MLA cache needs about 37 MiB of split-unit records on a 148-SM B200 (2 per cluster of
+ * 2 CTAs, 64 heads x 515 floats each per CTA), a GQA cache about 2.5 MB. */
+#define HELIX_NOALLOC_SCRATCH_BYTES (48u << 20)
 helix_status helix_attn_partial_noalloc(const helix_kv_cache* cache, const void* q,
                                         int32_t num_q_heads, float softmax_scale,
                                         float* o_partial, float* lse, helix_stream_t stream);

@@ -329,7 +329,7 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
     m.shard_lens = c->shard_lens;
     m.o_part = o_partial;
     m.lse = lse;
-    m.q = static_cast<const uint16_t*>(q);
+    m.pool = static_cast<const uint8_t*>(c->k_pool);
     m.tickets = reinterpret_cast<int32_t*>(workspace);
     m.seg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.ticket_bytes +
                                      plan.gticket_bytes);
@@ -339,13 +339,16 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
     m.max_pages = c->max_pages_per_shard;
     m.num_pages = c->num_pages;
     m.scale_log2 = softmax_scale * 1.4426950408889634f;
-    // latent pool as [pages * 64 rows][576], boxes of 64 columns x 64 rows; q as [B * 128][576],
-    // boxes of 64 columns x 128 rows; 128-byte swizzle for the tensor-core operand layout
-    CUtensorMap tmC, tmQ;
+    // latent pool as [pages * 64 rows][576]: boxes of 64 columns x 64 rows (one chunk of a page,
+    // the score operand) and 64 columns x 32 rows (value operand); q as [B * 128][576], boxes of
+    // 64 columns x 64 rows (one CTA's heads); 128-byte swizzle for the tensor-core operand layout
+    CUtensorMap tmC, tmV, tmQ;
     if (!encode_rows_map(&tmC, c->k_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
                          (uint64_t)c->num_pages * 64, 64, 64) ||
+        !encode_rows_map(&tmV, c->k_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
+                         (uint64_t)c->num_pages * 64, 64, 32) ||
         !encode_rows_map(&tmQ, const_cast<void*>(q), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
-                         (uint64_t)c->batch * 128, 64, 128))
+                         (uint64_t)c->batch * 128, 64, 64))
       return HELIX_ERR_CUDA;
     // request ranges of at most plan.max_units units each, one after another on the stream
     // (they share the workspace; the unit tickets are back at zero after each launch)
@@ -353,7 +356,7 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
     for (int b = b_begin; b < b_end; b += per) {
       m.u0 = b * units_per_request;
       m.units = (min(b_end, b + per) - b) * units_per_request;
-      st = mla_partial_launch(tmC, tmQ, m, plan.grid, stream);
+      st = mla_partial_launch(tmC, tmV, tmQ, m, plan.grid, stream);
       if (st != HELIX_OK) return st;
     }
     return HELIX_OK;

@@ -50,9 +50,9 @@ struct MlaParams {
   const int32_t* shard_lens;  // [kvp][B]
   float* o_part;              // [kvp][B][128][512]
   float* lse;                 // [kvp][B][128]
-  const uint16_t* q;          // bf16 [B][128][576] (also read through the q tensor map)
+  const uint8_t* pool;        // bf16 [pages * 64][576] (also read through the tensor maps)
   int32_t* tickets;           // [units][2], zero between launches
-  float* seg;                 // [clusters][2 slots][2 halves][record]
+  float* seg;                 // [clusters][2 slots][2 CTAs][record]
   uint32_t* err;              // may be null
   int B, kvp, max_pages, num_pages, units;
   int u0;                     // first unit of this launch (a request boundary)
@@ -60,8 +60,9 @@ struct MlaParams {
 };
 size_t mla_partial_smem_bytes(int units);
 size_t mla_segment_record_floats();
-helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmQ,
-                                const MlaParams& p, int grid, cudaStream_t stream);
+helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmV,
+                                const CUtensorMap& tmQ, const MlaParams& p, int grid,
+                                cudaStream_t stream);
 
 // Append: copies the new tokens' rows (and scales) into their pages.
 struct AppendParams {
