@@ -48,6 +48,22 @@ bool encode_rows_map(CUtensorMap* map, void* base, CUtensorMapDataType dt, int e
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The MLA latent pool (bf16 rows of 576) seen as a 3-D tensor [9 chunks][rows][64 columns]: the
+// chunk dimension has a stride of 128 bytes (one chunk of a row), so one box of 64 columns x 64 rows
+// x 2 chunks lands in shared memory as two consecutive 64-row chunk tiles in the 128-byte swizzled
+// layout the tensor cores read.
+bool encode_latent_chunks_map(CUtensorMap* map, void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {64, rows, 9};
+  const cuuint64_t strides[2] = {576 * 2, 64 * 2};
+  const cuuint32_t box[3] = {64, 64, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int device_sm_count(int* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -131,10 +147,10 @@ helix_status plan_partial(const helix_kv_cache* c, int num_q_heads, PartialPlan*
     int sms = 0, max_smem = 0;
     if (device_sm_count(&sms) != 0 || device_max_smem(&max_smem) != 0) return HELIX_ERR_CUDA;
     plan->units = c->batch * c->kvp;
-    // a launch keeps the prefix sums of its units in shared memory: a batch whose units do not
-    // fit is run as consecutive launches over request ranges
+    // a launch keeps three ints per unit (tile prefix sum, shard row, length) in shared memory:
+    // a batch whose units do not fit is run as consecutive launches over request ranges
     if (mla_partial_smem_bytes(0) > (size_t)max_smem) return HELIX_ERR_CAPACITY;
-    const size_t room = ((size_t)max_smem - mla_partial_smem_bytes(0)) / sizeof(int);
+    const size_t room = ((size_t)max_smem - mla_partial_smem_bytes(0)) / (3 * sizeof(int));
     const int fit = room < (size_t)plan->units ? (int)room : plan->units;
     plan->max_units = (fit / c->kvp) * c->kvp;
     if (plan->max_units < c->kvp) return HELIX_ERR_CAPACITY;
@@ -339,14 +355,11 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
     m.max_pages = c->max_pages_per_shard;
     m.num_pages = c->num_pages;
     m.scale_log2 = softmax_scale * 1.4426950408889634f;
-    // latent pool as [pages * 64 rows][576]: boxes of 64 columns x 64 rows (one chunk of a page,
-    // the score operand) and 64 columns x 32 rows (value operand); q as [B * 128][576], boxes of
-    // 64 columns x 64 rows (one CTA's heads); 128-byte swizzle for the tensor-core operand layout
-    CUtensorMap tmC, tmV, tmQ;
-    if (!encode_rows_map(&tmC, c->k_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
-                         (uint64_t)c->num_pages * 64, 64, 64) ||
-        !encode_rows_map(&tmV, c->k_pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
-                         (uint64_t)c->num_pages * 64, 64, 32) ||
+    // latent pool as [9 chunks][pages * 64 rows][64 columns]: boxes of two chunks of a page (a
+    // score slot, or a value slot of 128 columns); q as [B * 128][576], boxes of 64 columns x 64
+    // rows (one CTA's heads); 128-byte swizzle for the tensor-core operand layout
+    CUtensorMap tmC, tmQ;
+    if (!encode_latent_chunks_map(&tmC, c->k_pool, (uint64_t)c->num_pages * 64) ||
         !encode_rows_map(&tmQ, const_cast<void*>(q), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
                          (uint64_t)c->batch * 128, 64, 64))
       return HELIX_ERR_CUDA;
@@ -356,7 +369,7 @@ helix_status partial_impl(const helix_kv_cache* c, const void* q, int32_t num_q_
     for (int b = b_begin; b < b_end; b += per) {
       m.u0 = b * units_per_request;
       m.units = (min(b_end, b + per) - b) * units_per_request;
-      st = mla_partial_launch(tmC, tmV, tmQ, m, plan.grid, stream);
+      st = mla_partial_launch(tmC, tmQ, m, plan.grid, stream);
       if (st != HELIX_OK) return st;
     }
     return HELIX_OK;

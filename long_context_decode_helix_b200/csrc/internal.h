@@ -60,9 +60,8 @@ struct MlaParams {
 };
 size_t mla_partial_smem_bytes(int units);
 size_t mla_segment_record_floats();
-helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmV,
-                                const CUtensorMap& tmQ, const MlaParams& p, int grid,
-                                cudaStream_t stream);
+helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmQ,
+                                const MlaParams& p, int grid, cudaStream_t stream);
 
 // Append: copies the new tokens' rows (and scales) into their pages.
 struct AppendParams {

@@ -22,19 +22,22 @@
 //   * O += P V per tile, M = 128 heads (64 per SM), N = 256 value columns per MMA (each CTA
 //     supplies 128 of them: CTA r the 64-column chunks 2r, 2r + 1 of each 256-column block), K =
 //     128 tokens. P is written to shared memory by the softmax warps (the A operand, K-major);
-//     V is read again from L2 into the ring (MN-major), two 64-column chunks x 32 tokens per slot.
-// Operands stream through one ring of 8 KiB shared-memory slots in a fixed order that both CTAs'
-// producers and the MMA issuer walk together: the nine 64-column chunks of tile i's pages, then the
-// eight value slots of tile i - 1 (its P V runs after the scores of tile i, so the softmax of tile
-// i - 1 overlaps them). Every TMA load of either CTA completes on CTA 0's barrier of its slot; the
-// MMA's commits reach both CTAs (tcgen05.commit multicast). No TMA load uses cluster multicast.
+//     V is read again from L2 into the value ring (MN-major), two 64-column chunks x 64 tokens.
+// Operands stream through two rings of 16 KiB shared-memory slots, one per operand, each filled by
+// a producer warp in both CTAs: the score ring takes this CTA's page of each tile as five slots of
+// two 64-column chunks (one 3-D TMA box each; the fifth holds chunk 8 and zeros), the value ring
+// takes, per column block j and page, this CTA's two 64-column chunks of that page (read again,
+// from L2). Every TMA load of either CTA completes on CTA 0's barrier of its slot; the MMAs'
+// commits reach both CTAs (tcgen05.commit multicast). No TMA load uses cluster multicast.
 //
-// Warps: 0-3 softmax / epilogue, 4 score-operand producer and 7 value-operand producer (both
-// CTAs), 5 score-MMA issuer (CTA 0) and TMEM allocator, 6 P V-MMA issuer (CTA 0); each producer
-// feeds its issuer through a ring of its own. Softmax thread l reads TMEM lane l: lane l < 64 holds head l's scores of the first
-// page of the tile, lane 64 + l the same head's scores of the second page (the two-SM layout of an
-// M = 64-per-SM accumulator); the two threads of a head combine their row maxima through shared
-// memory. The tensor pipe computes the scores of tile i + 1 while the softmax works on tile i, and
+// Issue: a thread issuing a pair-wide tcgen05.mma is busy for longer than the tensor pipe needs
+// for these shapes, so three threads of CTA 0 issue: two take the first / second half of the
+// k-steps of every chunk into two score accumulators (the softmax adds them), the third issues
+// P V. They and the producers have the low warp ids; warps 4-7 are the softmax / epilogue warps.
+// Softmax thread l reads TMEM lane l: lane l < 64 holds head l's scores of the first page of the
+// tile, lane 64 + l the same head's scores of the second page (the two-SM layout of an M =
+// 64-per-SM accumulator); the two threads of a head combine their row maxima through shared
+// memory. The tensor pipe computes the scores of tile i + 1 while the softmax works on tile i;
 // the scores and P each have two buffers. The reference maximum moves lazily (only when a row
 // maximum exceeds it by more than 8 in base-2 units), so weights stay below 2^8 and the TMEM
 // rescale of O is rare; the logit scale is applied inside the exponent.
@@ -59,14 +62,22 @@ constexpr int kD = 576, kDV = 512;
 constexpr int kPage = 64;                // tokens per page (and per CTA per tile)
 constexpr int kTile = 2 * kPage;         // tokens per tile of the pair
 constexpr int kChunks = 9;               // 64-column chunks of a latent row
-constexpr int kSlot = 8192;              // ring slot bytes
-constexpr int kRingQ = 8;                // score-operand ring slots (page chunks)
-constexpr int kRingV = 6;                // value-operand ring slots
+constexpr int kSlot = 8192;              // one 64-column chunk of a page (64 rows x 128 B)
+constexpr int kQSlot = 2 * kSlot;        // score ring slot: two chunks of a page
+constexpr int kRingQ = 4;                // score-operand ring slots
+constexpr int kQSlotsPerTile = 5;        // chunks (0,1) (2,3) (4,5) (6,7) (8,-)
+constexpr int kVSlot = 2 * kSlot;        // value ring slot: 128 value columns of one page
+constexpr int kRingV = 3;                // value-operand ring slots
 constexpr int kQBytes = kChunks * kHc * 128;  // 72 KiB
 constexpr int kPBytes = 2 * kHc * 128;        // one tile's P: two 64-token K-chunks, 16 KiB
 constexpr uint32_t kOCol = 0, kSCol = 256, kTmemCols = 512;
-constexpr int kProducerWarp = 4, kMmaWarp = 5, kPvWarp = 6, kValueWarp = 7;
-constexpr int kThreads = 8 * 32;
+// Warp roles. The MMA issuers and the producers take the low warp ids: when a softmax warp and one
+// of them are both ready on an SM sub-partition, the scheduler was measured to favour the older
+// warp, and a softmax warp with ready arithmetic otherwise starves a thread issuing tcgen05.mma.
+// Warps 4-7 are the softmax warps (warp w reads TMEM lanes 32 (w % 4) .. + 31).
+constexpr int kMmaWarp2 = 0, kMmaWarp = 1, kPvWarp = 2, kValueWarp = 3, kSoftmaxWarp0 = 4,
+              kProducerWarp = 8;
+constexpr int kThreads = 9 * 32;
 constexpr int kRec = kHc * (kDV + 3);    // floats per segment record (this CTA's heads)
 constexpr float kLazy = 8.f;             // base-2 headroom before the reference maximum moves
 constexpr int kPf = 2;                   // tiles whose pages are fetched into L2 ahead of the ring
@@ -77,13 +88,13 @@ struct MlaTail {
   uint64_t empty_q[kRingQ];  // both: the MMAs that read the slot are done
   uint64_t full_v[kRingV];   // the same for the value ring
   uint64_t empty_v[kRingV];
-  uint64_t s_full[2];      // both: the scores of a tile are in TMEM
+  uint64_t s_full[2];      // both: the scores of a tile are in TMEM (both score issuers)
   uint64_t s_empty[2];     // CTA 0: the 4 softmax warps of each CTA read them
   uint64_t p_full[2];      // CTA 0: the 4 softmax warps of each CTA wrote P (and rescaled O)
   uint64_t p_empty[2];     // both: P V of the tile is done
   uint64_t q_full;         // CTA 0: its producer's arrival and both CTAs' q bytes
-  uint64_t q_empty;        // both: the last score MMA of a unit is done
-  uint64_t mma_done;       // both: every MMA issued by either thread has completed
+  uint64_t q_empty;        // both: the last score MMAs of a unit (both issuers) are done
+  uint64_t mma_done;       // both: every MMA issued by the three issuers has completed
   float xmax[2][kHeads];   // [tile parity][lane]: row maxima of the two token halves
   float xl[kHeads];        // [lane]: row sums of the two halves at a segment end
   int pid[kPid][2];        // producer only: page ids (or -1) of the two pages of a tile
@@ -93,7 +104,8 @@ struct MlaTail {
 };
 
 constexpr size_t kSmemFixed =
-    1024 + kQBytes + 2 * kPBytes + (size_t)(kRingQ + kRingV) * kSlot + sizeof(MlaTail);
+    1024 + kQBytes + 2 * kPBytes + (size_t)kRingQ * kQSlot + (size_t)kRingV * kVSlot +
+    sizeof(MlaTail);
 
 // ------------------------------------------------------------------------------------------------
 // cluster, mbarrier and tcgen05 helpers
@@ -146,6 +158,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// The same for a 3-D box (the latent pool seen as [chunk][row][64 columns]).
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map, int32_t x,
+                                                 int32_t y, int32_t z, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
+      : "memory");
+}
+// Brings `bytes` (a multiple of 16) of global memory at a 16-byte aligned address into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -169,6 +195,25 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
       " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
       : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane; the registers are valid after
+// tmem_wait_ld()
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 // 32 consecutive fp32 columns of this thread's TMEM lane
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -237,17 +282,18 @@ struct TileAt {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_partial_kernel(const __grid_constant__ CUtensorMap tmC,
-                       const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmQ, const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* q_s = smem;                      // [9 chunks][64 rows][128 B]
   uint8_t* p_s = q_s + kQBytes;             // [2 groups][2 token chunks][64 rows][128 B]
-  uint8_t* ring_q = p_s + 2 * kPBytes;      // [kRingQ][8 KiB]: page chunks (score operand)
-  uint8_t* ring_v = ring_q + (size_t)kRingQ * kSlot;  // [kRingV][8 KiB]: value operand
-  MlaTail* tail = reinterpret_cast<MlaTail*>(ring_v + (size_t)kRingV * kSlot);
-  int* pre = reinterpret_cast<int*>(tail + 1);
+  uint8_t* ring_q = p_s + 2 * kPBytes;      // [kRingQ][2 chunks][64 rows][128 B]: score operand
+  uint8_t* ring_v = ring_q + (size_t)kRingQ * kQSlot;  // [kRingV][2 chunks][64 rows][128 B]
+  MlaTail* tail = reinterpret_cast<MlaTail*>(ring_v + (size_t)kRingV * kVSlot);
+  int* pre = reinterpret_cast<int*>(tail + 1);  // [U + 1]: first tile of each unit
+  int* urow = pre + (p.units + 1);               // [U]: s * B + b, the unit's shard_lens index
+  int* ulen = urow + p.units;                    // [U]: the unit's token count (capped)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();
@@ -264,26 +310,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       len = p.max_pages * kPage;
     }
     pre[u + 1] = len > 0 ? (len + kTile - 1) / kTile : 0;
+    urow[u] = s * p.B + b;
+    ulen[u] = max(len, 0);
   }
   if (tid == 0) {
     pre[0] = 0;
     for (int i = 0; i < kRingQ; ++i) {
-      mbar_init(&tail->full_q[i], 1);  // CTA 0's producer, with both CTAs' bytes
-      mbar_init(&tail->empty_q[i], 1);
+      mbar_init(&tail->full_q[i], 1);   // CTA 0's producer, with both CTAs' bytes
+      mbar_init(&tail->empty_q[i], 2);  // the commits of both score issuers
     }
     for (int i = 0; i < kRingV; ++i) {
       mbar_init(&tail->full_v[i], 1);
       mbar_init(&tail->empty_v[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&tail->s_full[i], 1);
+      mbar_init(&tail->s_full[i], 2);  // the commits of both score issuers
       mbar_init(&tail->s_empty[i], 8);  // the 4 softmax warps of each CTA
       mbar_init(&tail->p_full[i], 8);
       mbar_init(&tail->p_empty[i], 1);
     }
     mbar_init(&tail->q_full, 1);
-    mbar_init(&tail->q_empty, 1);
-    mbar_init(&tail->mma_done, 2);  // both issuing threads' final commits
+    mbar_init(&tail->q_empty, 2);
+    mbar_init(&tail->mma_done, 3);  // the three issuing threads' final commits
     tail->flag = 0;
     tail->abort_ = 0;
     fence_mbar_init();
@@ -323,8 +371,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // units with no tokens: O_s = 0, lse_s = -inf (this CTA's heads)
   for (int u = pair; u < U; u += npairs) {
     if (pre[u + 1] != pre[u]) continue;
-    const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
-    const size_t row0 = ((size_t)s * p.B + b) * kHeads + (size_t)rank * kHc;
+    const size_t row0 = (size_t)urow[u] * kHeads + (size_t)rank * kHc;
     for (int i = tid; i < kHc * kDV; i += kThreads) p.o_part[row0 * kDV + i] = 0.f;
     for (int i = tid; i < kHc; i += kThreads) p.lse[row0 + i] = -INFINITY;
   }
@@ -345,10 +392,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   // page id of local page lp of unit u, or -1 (past the shard's pages, or outside the pool)
   auto page_of = [&](int u, int lp, bool report) -> int {
-    const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
-    const int len = min(p.shard_lens[s * p.B + b], p.max_pages * kPage);
-    if (lp * kPage >= len) return -1;
-    const int pg = __ldg(p.page_table + ((size_t)s * p.B + b) * p.max_pages + lp);
+    if (lp * kPage >= ulen[u]) return -1;
+    const int pg = __ldg(p.page_table + (size_t)urow[u] * p.max_pages + lp);
     if (pg < 0 || pg >= p.num_pages) {
       if (report) raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
       return -1;
@@ -395,9 +440,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ============================ score-operand producer (both CTAs) =============================
-    // For each tile, the nine 64-column chunks of this CTA's page; q of a new unit's request. Page
-    // ids are read kPf tiles ahead (lanes 0 and 1 take the tile's two pages) and this CTA's page is
-    // brought into L2 then, so the ring's loads find it there.
+    // For each tile, this CTA's page in five slots of two 64-column chunks (one 3-D TMA each; the
+    // fifth holds chunk 8 and zeros); q of a new unit's request. Page ids are used kPf tiles ahead
+    // (lanes 0 and 1 take the tile's two pages) to bring this CTA's page into L2, so the ring's
+    // loads find it there; their global loads are issued one tile before they are needed.
     if (active) {
       if (lane == 0) {
         prefetch_tensormap(&tmC);
@@ -407,40 +453,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool dead = false;
       TileAt at_r;
       at_r.u = u_first;
-      auto resolve = [&](long long t) {
+      int r_raw = -1, r_len = 0, r_lp = 0;  // loads in flight for the next tile to resolve
+      auto issue_ids = [&](long long t) {  // starts the loads of tile t's page ids (no wait)
         const long long g = g_begin + t;
         at_r.seek(pre, g);
-        const int tt = (int)(g - pre[at_r.u]);
+        const int u = at_r.u;
+        r_lp = 2 * (int)(g - pre[u]) + (lane & 1);
+        r_len = ulen[u];
+        r_raw = r_lp < p.max_pages ? __ldg(p.page_table + (size_t)urow[u] * p.max_pages + r_lp)
+                                   : -1;
+      };
+      auto finish_ids = [&](long long t) {  // page ids of tile t into the queue; L2 prefetch
         int pg = -1;
-        if (lane < 2) {
-          pg = page_of(at_r.u, 2 * tt + lane, true);
-          tail->pid[t % kPid][lane] = pg;
+        if (r_lp * kPage < r_len) {
+          if (r_raw < 0 || r_raw >= p.num_pages) {
+            if (lane < 2) raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
+          } else {
+            pg = r_raw;
+          }
         }
-        pg = __shfl_sync(0xffffffffu, pg, (int)rank);
-        if (lane == 0 && pg >= 0)
-          for (int c = 0; c < kChunks; ++c) tma_prefetch_l2_2d(&tmC, 64 * c, pg * kPage);
+        if (lane < 2) tail->pid[t % kPid][lane] = pg;
+        const int mine = __shfl_sync(0xffffffffu, pg, (int)rank);
+        if (lane == 0 && mine >= 0)
+          bulk_prefetch_l2(p.pool + (size_t)mine * kPage * (kD * 2), kPage * kD * 2);
         __syncwarp();
       };
       TileAt at_q;
       at_q.u = u_first;
       int cur = -1, qcount = 0;
-      for (long long t = 0; t < kPf && t < n_tiles; ++t) resolve(t);
+      for (long long t = 0; t < kPf && t < n_tiles; ++t) {
+        issue_ids(t);
+        finish_ids(t);
+      }
+      if (kPf < n_tiles) issue_ids(kPf);
       for (long long i = 0; i < n_tiles && !dead; ++i) {
         if (*(volatile int*)&tail->abort_) { dead = true; break; }
-        if (i + kPf < n_tiles) resolve(i + kPf);
+        if (i + kPf < n_tiles) {
+          finish_ids(i + kPf);
+          if (i + kPf + 1 < n_tiles) issue_ids(i + kPf + 1);
+        }
         const long long g = g_begin + i;
         at_q.seek(pre, g);
         const int u = at_q.u;
         if (u != cur) {  // this CTA's 64 heads of q for the unit's request, once the previous
                          // unit's score MMAs are done with the buffer. It goes before the tile's
-                         // chunks: the issuer takes no chunk of the unit before q, and the ring is
-                         // shorter than a tile's nine chunks.
+                         // chunks: the issuers take no chunk of the unit before q, and the ring is
+                         // shorter than a tile.
           if (qcount > 0) {
             const bool ok = mbar_wait_pair(&tail->q_empty, (qcount - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) { dead = true; break; }
           }
           if (lane == 0) {
-            const int b = (u + p.u0) / p.kvp;
+            const int b = urow[u] % p.B;
             if (rank == 0) mbar_arrive_expect_tx(&tail->q_full, 2 * kQBytes);
             for (int c = 0; c < kChunks; ++c)
               tma_load_2d_pair(q_s + c * kHc * 128, &tmQ, 64 * c, b * kHeads + (int)rank * kHc,
@@ -451,12 +515,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         const int pg = tail->pid[i % kPid][rank];
         const int y = pg < 0 ? oob_row : pg * kPage;
-        for (int c = 0; c < kChunks; ++c) {
+        for (int sl = 0; sl < kQSlotsPerTile; ++sl) {
           const int k = acquire(rq);
           if (k < 0) { dead = true; break; }
           if (lane == 0) {
-            if (rank == 0) mbar_arrive_expect_tx(&tail->full_q[k], 2 * kSlot);
-            tma_load_2d_pair(ring_q + (size_t)k * kSlot, &tmC, 64 * c, y, lead_full_q0 + 8u * k);
+            if (rank == 0) mbar_arrive_expect_tx(&tail->full_q[k], 2 * kQSlot);
+            tma_load_3d_pair(ring_q + (size_t)k * kQSlot, &tmC, 0, y, 2 * sl, lead_full_q0 + 8u * k);
           }
         }
       }
@@ -467,12 +531,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kValueWarp) {
     // ============================ value-operand producer (both CTAs) =============================
-    // For each tile, column block j and 32-token chunk kc: this CTA's two 64-column chunks
-    // (4 j + 2 rank, + 1) of the tile's tokens 32 kc .. 32 kc + 31 (read again, from L2: both
-    // pages of the tile were just loaded for the scores). The next tile's page ids are read while
-    // this tile's slots are filled.
+    // For each tile, column block j and page `half` of the tile: this CTA's two 64-column chunks
+    // (4 j + 2 rank, + 1) of the page's 64 tokens, read again (from L2: both pages of the tile were
+    // just loaded for the scores). The next tile's page ids are read while this tile's slots fill.
     if (active) {
-      if (lane == 0) prefetch_tensormap(&tmV);
+      if (lane == 0) prefetch_tensormap(&tmC);
       Ring rv{tail->full_v, tail->empty_v, kRingV};
       bool dead = false;
       TileAt at;
@@ -495,44 +558,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int u = at.u, tt = (int)(g - pre[u]);
         if (u != len_cur_u) {
           len_cur_u = u;
-          const int s_ = (u + p.u0) % p.kvp, b_ = (u + p.u0) / p.kvp;
-          len = min(p.shard_lens[s_ * p.B + b_], p.max_pages * kPage);
+          len = ulen[u];
         }
         for (int j = 0; j < 2 && !dead; ++j) {
-          for (int kc = 0; kc < 4; ++kc) {
+          for (int half = 0; half < 2; ++half) {
             const int k = acquire(rv);
             if (k < 0) { dead = true; break; }
-            const int half = kc >> 1, r0 = (kc & 1) * 32;
             const int pg = half ? pgB : pgA;
-            const int nvalid = min(max(len - (2 * tt + half) * kPage - r0, 0), 32);
-            uint8_t* slot = ring_v + (size_t)k * kSlot;
+            const int nvalid = min(max(len - (2 * tt + half) * kPage, 0), kPage);
+            uint8_t* slot = ring_v + (size_t)k * kVSlot;
             const int cb = 4 * j + 2 * (int)rank;
             // CTA 0 expects both CTAs' bytes of the slot
-            if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&tail->full_v[k], 2 * kSlot);
-            if (pg < 0 || nvalid == 0 || nvalid == 32) {
-              // whole box of history rows, or nothing of the history (zeros from past the pool)
+            if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&tail->full_v[k], 2 * kVSlot);
+            if (pg < 0 || nvalid == 0 || nvalid == kPage) {
+              // the whole page, or nothing of the history (zeros from past the pool)
               if (lane == 0) {
-                const int y = (pg < 0 || nvalid == 0) ? oob_row : pg * kPage + r0;
-                tma_load_2d_pair(slot, &tmV, 64 * cb, y, lead_full_v0 + 8u * k);
-                tma_load_2d_pair(slot + 4096, &tmV, 64 * (cb + 1), y, lead_full_v0 + 8u * k);
+                const int y = (pg < 0 || nvalid == 0) ? oob_row : pg * kPage;
+                tma_load_3d_pair(slot, &tmC, 0, y, cb, lead_full_v0 + 8u * k);
               }
             } else {
-              // the last, partial 32 rows of a shard: rows of the history are copied, rows past it
+              // the last, partial page of a shard: rows of the history are copied, rows past it
               // are zeroed (a zero weight times a non-finite stale value would not be zero), in
               // the 128-byte swizzled layout TMA writes
-              for (int e = lane; e < 2 * 32 * 8; e += 32) {
-                const int sb = e >> 8, r = (e >> 3) & 31, un = e & 7;
+              for (int e = lane; e < 2 * kPage * 8; e += 32) {
+                const int sb = e >> 9, r = (e >> 3) & (kPage - 1), un = e & 7;
                 uint4 v = make_uint4(0, 0, 0, 0);
                 if (r < nvalid)
                   v = __ldg(reinterpret_cast<const uint4*>(
-                      p.pool + ((size_t)pg * kPage + r0 + r) * (kD * 2) + (64 * (cb + sb) + 8 * un) * 2));
-                *reinterpret_cast<uint4*>(slot + sb * 4096 + r * 128 + ((un ^ (r & 7)) << 4)) = v;
+                      p.pool + ((size_t)pg * kPage + r) * (kD * 2) + (64 * (cb + sb) + 8 * un) * 2));
+                *reinterpret_cast<uint4*>(slot + sb * kSlot + r * 128 + ((un ^ (r & 7)) << 4)) = v;
               }
               fence_proxy_async_smem();  // the generic-proxy stores before the MMA's reads
               __syncwarp();
               if (lane == 0) {
                 asm volatile("fence.acq_rel.cluster;" ::: "memory");
-                complete_tx_remote(lead_full_v0 + 8u * k, kSlot);
+                complete_tx_remote(lead_full_v0 + 8u * k, kVSlot);
               }
             }
           }
@@ -543,23 +603,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *(volatile int*)&tail->abort_ = 1;
       }
     }
-  } else if (warp == kMmaWarp || warp == kPvWarp) {
-    // ======================== MMA issuers (CTA 0: one thread in each warp) ========================
-    // The score MMAs and the P V MMAs are issued by two threads, each fed by its own ring: issuing
-    // a tcgen05.mma costs its thread tens of cycles, more than the tensor pipe needs for one of
-    // these MMAs, so one thread issuing both kinds would leave the pipe idle half the time.
-    const bool qk = warp == kMmaWarp;
+  } else if (warp == kMmaWarp || warp == kMmaWarp2 || warp == kPvWarp) {
+    // ====================== MMA issuers (CTA 0: one thread in each of three warps) ===============
+    // Issuing a pair-wide tcgen05.mma occupies its thread for longer than the tensor pipe needs to
+    // execute one of these shapes (64 x 128 x 16 and 64 x 256 x 16 per SM), so one thread cannot
+    // keep the pipe busy. Three threads on three SM sub-partitions issue: score issuer `role` 0 / 1
+    // takes the first / second half of the k-steps of every 64-column chunk into its own score
+    // accumulator (the softmax adds the two), the third issues P V. Descriptors are formed once and advanced by
+    // constants, so little but the MMAs themselves runs between them.
+    const int role = warp == kMmaWarp ? 0 : warp == kMmaWarp2 ? 1 : 2;
     if (rank == 0 && lane == 0 && active) {
       constexpr uint32_t idQK = make_idesc(128, kTile, false);
       constexpr uint32_t idPV = make_idesc(128, 256, true);
-      const uint32_t qbase = smem_u32(q_s), pbase = smem_u32(p_s);
-      const uint32_t rq_base = smem_u32(ring_q), rv_base = smem_u32(ring_v);
       bool dead = false;
       TileAt at;
       at.u = u_first;
-      if (qk) {
-        Ring rq{tail->full_q, tail->empty_q, kRingQ};
+      if (role < 2) {
+        // S_role(i) = the k-steps kk = 2 role, 2 role + 1 of every 64-column chunk c of tile i:
+        // sum of q[:, 64c + 16kk : +16] C[:, 64c + 16kk : +16]^T. Both threads wait for every
+        // slot in ring order (a thread that skipped slots could mistake an old phase of a slot for
+        // the one it wants: the waits go by phase parity) and each commits the slot's release
+        // (count 2). Slot sl of tile i is ring position 5 i + sl; a k-step of 16 columns advances
+        // the start address 32 B (2 descriptor units) inside the 128-byte swizzled rows; chunk
+        // c + 1 of a slot follows chunk c at 8 KiB.
+        const uint64_t qd = smem_desc(smem_u32(q_s), 16, 1024) + (uint64_t)(4 * role);
+        const uint64_t rd = smem_desc(smem_u32(ring_q), 16, 1024) + (uint64_t)(4 * role);
         int cur = -1, qcount = 0;
+        uint32_t pos = 0;  // ring position of the next slot
         for (long long i = 0; i < n_tiles && !dead; ++i) {
           if (*(volatile int*)&tail->abort_) { dead = true; break; }
           const long long g = g_begin + i;
@@ -569,23 +639,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             cur = at.u;
             ++qcount;
           }
-          if (i >= 2 &&
-              !mbar_wait_pair(&tail->s_empty[i & 1], (uint32_t)(((i - 2) >> 1) & 1))) {
-            dead = true;
-            break;
+          if (i >= 2) {
+            if (!mbar_wait_pair(&tail->s_empty[i & 1], (uint32_t)(((i - 2) >> 1) & 1))) {
+              dead = true;
+              break;
+            }
+            tc_fence_after();  // the softmax's TMEM reads of the buffer came first
           }
-          // S(i) = q C^T: 9 chunks x 4 k-steps of 16 columns; a k-step advances the start address
-          // 32 B inside the 128-byte swizzled rows
-          const uint32_t d_s = tmem + kSCol + (uint32_t)(i & 1) * (kTile / 2);
-          for (int c = 0; c < kChunks; ++c) {
-            const int ks = take(rq);
-            if (ks < 0) { dead = true; break; }
-            tc_fence_after();
+          const uint32_t d_s = tmem + kSCol + (uint32_t)(i & 1) * kTile + (uint32_t)role * (kTile / 2);
+          for (int sl = 0; sl < kQSlotsPerTile; ++sl, ++pos) {
+            const int ks = (int)(pos % kRingQ);
+            if (!mbar_wait_pair(&tail->full_q[ks], (uint32_t)((pos / kRingQ) & 1))) {
+              dead = true;
+              break;
+            }
+            const uint64_t bs = rd + (uint64_t)((ks * kQSlot) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t a = smem_desc(qbase + (uint32_t)c * (kHc * 128) + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc(rq_base + (uint32_t)ks * kSlot + kk * 32, 16, 1024);
-              tc_mma_pair(d_s, a, bd, idQK, (c | kk) != 0);
+            for (int cc = 0; cc < 2; ++cc) {
+              const int c = 2 * sl + cc;
+              if (c >= kChunks) break;
+              const uint64_t a = qd + (uint64_t)((c * (kHc * 128)) >> 4);
+              const uint64_t bd = bs + (uint64_t)((cc * kSlot) >> 4);
+              tc_mma_pair(d_s, a, bd, idQK, c != 0);
+              tc_mma_pair(d_s, a + 2, bd + 2, idQK, true);
             }
             tc_commit_pair(&tail->empty_q[ks]);
           }
@@ -595,6 +671,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (g + 1 == g_end || g + 1 == pre[at.u + 1]) tc_commit_pair(&tail->q_empty);
         }
       } else {
+        // O[:, 256 j : 256 j + 256] += P V per page `half` of the tile: 4 k-steps of 16 tokens.
+        // A = P of this CTA's 64 heads (K-major, page `half` is a 64-token chunk, 32 B per step);
+        // B = V slot (MN-major: two 64-column sub-blocks 8 KiB apart, 8-token groups 1 KiB apart,
+        // 16 tokens = 2 KiB per step).
+        const uint64_t pd = smem_desc(smem_u32(p_s), 16, 1024);
+        const uint64_t vd = smem_desc(smem_u32(ring_v), kSlot, 1024);
         Ring rv{tail->full_v, tail->empty_v, kRingV};
         for (long long t = 0; t < n_tiles && !dead; ++t) {  // O += P V of tile t
           if (*(volatile int*)&tail->abort_) { dead = true; break; }
@@ -602,29 +684,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             dead = true;
             break;
           }
+          tc_fence_after();  // P (generic stores, proxy-fenced) and the O rescale came first
           const long long g = g_begin + t;
           at.seek(pre, g);
           const bool fresh = t == 0 || g == pre[at.u];  // first tile of a segment
-          tc_fence_after();
-          const uint32_t pb = pbase + (uint32_t)(t & 1) * kPBytes;
+          const uint64_t pt = pd + (uint64_t)(((uint32_t)(t & 1) * kPBytes) >> 4);
           for (int j = 0; j < 2 && !dead; ++j) {
-            for (int kc = 0; kc < 4; ++kc) {
+            for (int half = 0; half < 2; ++half) {
               const int ks = take(rv);
               if (ks < 0) { dead = true; break; }
-              tc_fence_after();
+              const uint64_t a = pt + (uint64_t)((half * (kHc * 128)) >> 4);
+              const uint64_t bd = vd + (uint64_t)((ks * kVSlot) >> 4);
 #pragma unroll
-              for (int s2 = 0; s2 < 2; ++s2) {
-                const int kt = 2 * kc + s2;  // 16-token step of the tile (0..7)
-                // A = P [64 heads x 16 tokens] per CTA, K-major: token chunk kt / 4, 32 B per step
-                const uint64_t a = smem_desc(pb + (uint32_t)(kt >> 2) * (kHc * 128) +
-                                                 (uint32_t)(kt & 3) * 32, 16, 1024);
-                // B = V [16 tokens x 128 columns] per CTA, MN-major: two 64-column sub-blocks
-                // 4 KiB apart, 8-token groups 1 KiB apart
-                const uint64_t bd = smem_desc(rv_base + (uint32_t)ks * kSlot + (uint32_t)s2 * 2048,
-                                              4096, 1024);
-                tc_mma_pair(tmem + kOCol + (uint32_t)j * 128, a, bd, idPV,
-                            !(fresh && kc == 0 && s2 == 0));
-              }
+              for (int kt = 0; kt < 4; ++kt)
+                tc_mma_pair(tmem + kOCol + (uint32_t)j * 128, a + 2 * kt, bd + 128 * kt, idPV,
+                            !(fresh && half == 0 && kt == 0));
               tc_commit_pair(&tail->empty_v[ks]);
             }
           }
@@ -643,10 +717,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ============================== softmax / epilogue warps =====================================
     // Thread lr (= TMEM lane lr) holds local head hl = lr % 64 and the 64 tokens of page half =
     // lr / 64 of each tile; the two threads of a head agree on its maximum through shared memory.
-    const int lr = tid;                 // TMEM lane of this thread (warps 0-3)
+    const int lr = tid - 32 * kSoftmaxWarp0;  // TMEM lane of this thread
     const int hl = lr & (kHc - 1);      // local head (row of this CTA's q)
     const int half = lr >> 6;           // which page of the tile this lane's scores belong to
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t lead_s_empty = map_rank(&tail->s_empty[0], 0);
     const uint32_t lead_p_full = map_rank(&tail->p_full[0], 0);
     const float sl2 = p.scale_log2;
@@ -659,23 +733,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
     TileAt at;
     at.u = u_first;
-    int len_u = 0, cur_u = -1;
+    // The shard length and this lane's page id of tile i + 1 are loaded while tile i is worked on
+    // (a page-table line is often no longer in L2 by the time it is needed).
+    TileAt at_n;
+    at_n.u = u_first;
+    int nx_raw = -1;
+    auto load_next = [&](long long t) {
+      const long long g = g_begin + t;
+      at_n.seek(pre, g);
+      const int u = at_n.u;
+      const int lp = 2 * (int)(g - pre[u]) + half;
+      nx_raw = lp < p.max_pages ? __ldg(p.page_table + (size_t)urow[u] * p.max_pages + lp) : -1;
+    };
+    if (n_tiles > 0) load_next(0);
     float sv[kPage];
     for (long long i = 0; i < n_tiles; ++i) {
       const long long g = g_begin + i;
       at.seek(pre, g);
       const int u = at.u;
-      if (u != cur_u) {
-        cur_u = u;
-        const int s_ = (u + p.u0) % p.kvp, b_ = (u + p.u0) / p.kvp;
-        len_u = min(p.shard_lens[s_ * p.B + b_], p.max_pages * kPage);
-      }
+      const int len_u = ulen[u], raw = nx_raw;  // raw: loaded during the previous tile
+      if (i + 1 < n_tiles) load_next(i + 1);
       const bool fresh = g == g_begin || g == pre[u];
       const bool seg_end = g + 1 == g_end || g + 1 == pre[u + 1];
-      const int s = (u + p.u0) % p.kvp, b = (u + p.u0) / p.kvp;
       const int tt = (int)(g - pre[u]);
       const int nvalid = min(max(len_u - (2 * tt + half) * kPage, 0), kPage);
-      const bool page_ok = nvalid > 0 && page_of(u, 2 * tt + half, false) >= 0;
+      const bool page_ok = nvalid > 0 && raw >= 0 && raw < p.num_pages;
       const int sb = (int)(i & 1);
       if (fresh) {  // a new segment: O starts over (its first P V overwrites the accumulator)
         m_ref = -INFINITY;
@@ -685,14 +767,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       dead = __any_sync(0xffffffffu, dead || *(volatile int*)&tail->abort_ != 0);
       wwait(&tail->s_full[sb], (uint32_t)((i >> 1) & 1));
       if (!dead) {
+        // S = S_0 + S_1, the accumulators of the two score issuers (64 columns each)
         tc_fence_after();
-        float v0[32], v1[32];
-        tmem_ld32(tl + kSCol + sb * (kTile / 2), v0);
-        tmem_ld32(tl + kSCol + sb * (kTile / 2) + 32, v1);
+        const uint32_t sa = tl + kSCol + (uint32_t)sb * kTile;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          sv[c] = v0[c];
-          sv[32 + c] = v1[c];
+        for (int h2 = 0; h2 < 2; ++h2) {
+          float v0[32], v1[32];
+          tmem_ld32_nowait(sa + 32 * h2, v0);
+          tmem_ld32_nowait(sa + kTile / 2 + 32 * h2, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sv[32 * h2 + c] = v0[c] + v1[c];
         }
         tc_fence_before();
       } else {
@@ -788,7 +873,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       named_barrier_sync(1, kHeads);
       const float M = m_ref;  // the reference O and both sums are relative to
       const float l_run = l_own + tail->xl[lr ^ 64];
-      const size_t orow = ((size_t)s * p.B + b) * kHeads + (size_t)rank * kHc + hl;
+      const size_t orow = (size_t)urow[u] * kHeads + (size_t)rank * kHc + hl;
       const bool whole = g_begin <= pre[u] && g + 1 == pre[u + 1];
       float* rec = nullptr;
       if (!whole) {
@@ -899,16 +984,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t mla_partial_smem_bytes(int units) { return kSmemFixed + (size_t)(units + 1) * sizeof(int); }
+size_t mla_partial_smem_bytes(int units) {
+  return kSmemFixed + (size_t)(3 * units + 1) * sizeof(int);  // pre, urow, ulen
+}
 size_t mla_segment_record_floats() { return kRec; }
 
-helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmV,
-                                const CUtensorMap& tmQ, const MlaParams& p, int grid,
-                                cudaStream_t stream) {
+helix_status mla_partial_launch(const CUtensorMap& tmC, const CUtensorMap& tmQ,
+                                const MlaParams& p, int grid, cudaStream_t stream) {
   const size_t smem = mla_partial_smem_bytes(p.units);
   if (allow_max_dynamic_smem(reinterpret_cast<const void*>(mla_partial_kernel)) != cudaSuccess)
     return HELIX_ERR_CUDA;
-  mla_partial_kernel<<<grid, kThreads, smem, stream>>>(tmC, tmV, tmQ, p);
+  mla_partial_kernel<<<grid, kThreads, smem, stream>>>(tmC, tmQ, p);
   return cudaGetLastError() == cudaSuccess ? HELIX_OK : HELIX_ERR_CUDA;
 }
 
