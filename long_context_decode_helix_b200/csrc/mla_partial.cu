@@ -271,12 +271,30 @@ __device__ __forceinline__ int cta_of(long long x, long long W, int G) {
   return (int)(((x + 1) * (long long)G - 1) / W);
 }
 
-// Where tile g of the cluster's range lies: its unit, its position in the unit and whether it
-// opens / closes a segment (a unit's tiles inside one cluster's range).
-struct TileAt {
-  int u = 0;
-  __device__ __forceinline__ void seek(const int* pre, long long g) {
-    while (pre[u + 1] <= g) ++u;
+// The unit that tile g of the cluster's range belongs to, with the unit's first tile, the first
+// tile past it, its shard row (s * B + b) and its token count kept in registers: they are read
+// from shared memory only when the unit changes.
+struct UnitCursor {
+  int u, first, next, row, len;
+  __device__ __forceinline__ void start(const int* pre, const int* urow, const int* ulen, int u0) {
+    u = u0;
+    first = pre[u];
+    next = pre[u + 1];
+    row = urow[u];
+    len = ulen[u];
+  }
+  // moves to the unit of tile g (g never decreases); true when the unit changed
+  __device__ __forceinline__ bool seek(const int* pre, const int* urow, const int* ulen,
+                                       long long g) {
+    if (g < next) return false;
+    do {
+      ++u;
+      first = next;
+      next = pre[u + 1];
+    } while (next <= g);
+    row = urow[u];
+    len = ulen[u];
+    return true;
   }
 };
 
@@ -390,16 +408,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     u_first = lo;
     while (pre[u_first + 1] <= g_begin) ++u_first;
   }
-  // page id of local page lp of unit u, or -1 (past the shard's pages, or outside the pool)
-  auto page_of = [&](int u, int lp, bool report) -> int {
-    if (lp * kPage >= ulen[u]) return -1;
-    const int pg = __ldg(p.page_table + (size_t)urow[u] * p.max_pages + lp);
-    if (pg < 0 || pg >= p.num_pages) {
-      if (report) raise_dev_error(p.err, HELIX_DEVERR_PAGE_ID);
-      return -1;
-    }
-    return pg;
-  };
   const uint32_t lead_full_q0 = map_rank(&tail->full_q[0], 0);
   const uint32_t lead_full_v0 = map_rank(&tail->full_v[0], 0);
   const uint32_t lead_q_full = map_rank(&tail->q_full, 0);
@@ -451,16 +459,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       Ring rq{tail->full_q, tail->empty_q, kRingQ};
       bool dead = false;
-      TileAt at_r;
-      at_r.u = u_first;
+      UnitCursor at_r;
+      at_r.start(pre, urow, ulen, u_first);
       int r_raw = -1, r_len = 0, r_lp = 0;  // loads in flight for the next tile to resolve
       auto issue_ids = [&](long long t) {  // starts the loads of tile t's page ids (no wait)
         const long long g = g_begin + t;
-        at_r.seek(pre, g);
-        const int u = at_r.u;
-        r_lp = 2 * (int)(g - pre[u]) + (lane & 1);
-        r_len = ulen[u];
-        r_raw = r_lp < p.max_pages ? __ldg(p.page_table + (size_t)urow[u] * p.max_pages + r_lp)
+        at_r.seek(pre, urow, ulen, g);
+        r_lp = 2 * (int)(g - at_r.first) + (lane & 1);
+        r_len = at_r.len;
+        r_raw = r_lp < p.max_pages ? __ldg(p.page_table + (size_t)at_r.row * p.max_pages + r_lp)
                                    : -1;
       };
       auto finish_ids = [&](long long t) {  // page ids of tile t into the queue; L2 prefetch
@@ -478,8 +485,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           bulk_prefetch_l2(p.pool + (size_t)mine * kPage * (kD * 2), kPage * kD * 2);
         __syncwarp();
       };
-      TileAt at_q;
-      at_q.u = u_first;
+      UnitCursor at_q;
+      at_q.start(pre, urow, ulen, u_first);
       int cur = -1, qcount = 0;
       for (long long t = 0; t < kPf && t < n_tiles; ++t) {
         issue_ids(t);
@@ -487,13 +494,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (kPf < n_tiles) issue_ids(kPf);
       for (long long i = 0; i < n_tiles && !dead; ++i) {
-        if (*(volatile int*)&tail->abort_) { dead = true; break; }
+        if ((i & 7) == 0 && *(volatile int*)&tail->abort_) { dead = true; break; }
         if (i + kPf < n_tiles) {
           finish_ids(i + kPf);
           if (i + kPf + 1 < n_tiles) issue_ids(i + kPf + 1);
         }
         const long long g = g_begin + i;
-        at_q.seek(pre, g);
+        at_q.seek(pre, urow, ulen, g);
         const int u = at_q.u;
         if (u != cur) {  // this CTA's 64 heads of q for the unit's request, once the previous
                          // unit's score MMAs are done with the buffer. It goes before the tile's
@@ -504,7 +511,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, ok)) { dead = true; break; }
           }
           if (lane == 0) {
-            const int b = urow[u] % p.B;
+            const int b = at_q.row % p.B;
             if (rank == 0) mbar_arrive_expect_tx(&tail->q_full, 2 * kQBytes);
             for (int c = 0; c < kChunks; ++c)
               tma_load_2d_pair(q_s + c * kHc * 128, &tmQ, 64 * c, b * kHeads + (int)rank * kHc,
@@ -538,28 +545,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) prefetch_tensormap(&tmC);
       Ring rv{tail->full_v, tail->empty_v, kRingV};
       bool dead = false;
-      TileAt at;
-      at.u = u_first;
-      int len_cur_u = -1, len = 0;
+      UnitCursor at, at_n;
+      at.start(pre, urow, ulen, u_first);
+      at_n = at;
       auto ids = [&](long long t) -> int {  // lane 0: page A, lane 1: page B of tile t
         const long long g = g_begin + t;
-        TileAt a2 = at;
-        a2.seek(pre, g);
-        const int tt = (int)(g - pre[a2.u]);
-        return lane < 2 ? page_of(a2.u, 2 * tt + lane, false) : -1;
+        at_n.seek(pre, urow, ulen, g);
+        const int lp = 2 * (int)(g - at_n.first) + lane;
+        if (lane >= 2 || lp * kPage >= at_n.len) return -1;
+        const int pg = __ldg(p.page_table + (size_t)at_n.row * p.max_pages + lp);
+        return (pg < 0 || pg >= p.num_pages) ? -1 : pg;
       };
       int nxt = n_tiles > 0 ? ids(0) : -1;
       for (long long t = 0; t < n_tiles && !dead; ++t) {
-        if (*(volatile int*)&tail->abort_) { dead = true; break; }
+        if ((t & 7) == 0 && *(volatile int*)&tail->abort_) { dead = true; break; }
         const int pgA = __shfl_sync(0xffffffffu, nxt, 0), pgB = __shfl_sync(0xffffffffu, nxt, 1);
         if (t + 1 < n_tiles) nxt = ids(t + 1);
         const long long g = g_begin + t;
-        at.seek(pre, g);
-        const int u = at.u, tt = (int)(g - pre[u]);
-        if (u != len_cur_u) {
-          len_cur_u = u;
-          len = ulen[u];
-        }
+        at.seek(pre, urow, ulen, g);
+        const int tt = (int)(g - at.first), len = at.len;
         for (int j = 0; j < 2 && !dead; ++j) {
           for (int half = 0; half < 2; ++half) {
             const int k = acquire(rv);
@@ -616,8 +620,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr uint32_t idQK = make_idesc(128, kTile, false);
       constexpr uint32_t idPV = make_idesc(128, 256, true);
       bool dead = false;
-      TileAt at;
-      at.u = u_first;
+      UnitCursor at;
+      at.start(pre, urow, ulen, u_first);
       if (role < 2) {
         // S_role(i) = the k-steps kk = 2 role, 2 role + 1 of every 64-column chunk c of tile i:
         // sum of q[:, 64c + 16kk : +16] C[:, 64c + 16kk : +16]^T. Both threads wait for every
@@ -631,9 +635,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int cur = -1, qcount = 0;
         uint32_t pos = 0;  // ring position of the next slot
         for (long long i = 0; i < n_tiles && !dead; ++i) {
-          if (*(volatile int*)&tail->abort_) { dead = true; break; }
+          if ((i & 7) == 0 && *(volatile int*)&tail->abort_) { dead = true; break; }
           const long long g = g_begin + i;
-          at.seek(pre, g);
+          at.seek(pre, urow, ulen, g);
           if (at.u != cur) {
             if (!mbar_wait_pair(&tail->q_full, (uint32_t)(qcount & 1))) { dead = true; break; }
             cur = at.u;
@@ -668,7 +672,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (dead) break;
           tc_commit_pair(&tail->s_full[i & 1]);
           // the last tile of a unit (or of the range) releases q for the next unit
-          if (g + 1 == g_end || g + 1 == pre[at.u + 1]) tc_commit_pair(&tail->q_empty);
+          if (g + 1 == g_end || g + 1 == at.next) tc_commit_pair(&tail->q_empty);
         }
       } else {
         // O[:, 256 j : 256 j + 256] += P V per page `half` of the tile: 4 k-steps of 16 tokens.
@@ -679,15 +683,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint64_t vd = smem_desc(smem_u32(ring_v), kSlot, 1024);
         Ring rv{tail->full_v, tail->empty_v, kRingV};
         for (long long t = 0; t < n_tiles && !dead; ++t) {  // O += P V of tile t
-          if (*(volatile int*)&tail->abort_) { dead = true; break; }
+          if ((t & 7) == 0 && *(volatile int*)&tail->abort_) { dead = true; break; }
           if (!mbar_wait_pair(&tail->p_full[t & 1], (uint32_t)((t >> 1) & 1))) {
             dead = true;
             break;
           }
           tc_fence_after();  // P (generic stores, proxy-fenced) and the O rescale came first
           const long long g = g_begin + t;
-          at.seek(pre, g);
-          const bool fresh = t == 0 || g == pre[at.u];  // first tile of a segment
+          at.seek(pre, urow, ulen, g);
+          const bool fresh = t == 0 || g == at.first;  // first tile of a segment
           const uint64_t pt = pd + (uint64_t)(((uint32_t)(t & 1) * kPBytes) >> 4);
           for (int j = 0; j < 2 && !dead; ++j) {
             for (int half = 0; half < 2; ++half) {
@@ -731,31 +735,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (dead) return;
       if (!__all_sync(0xffffffffu, mbar_wait_pair(bar, parity))) dead = true;
     };
-    TileAt at;
-    at.u = u_first;
-    // The shard length and this lane's page id of tile i + 1 are loaded while tile i is worked on
-    // (a page-table line is often no longer in L2 by the time it is needed).
-    TileAt at_n;
-    at_n.u = u_first;
+    UnitCursor at, at_n;
+    at.start(pre, urow, ulen, u_first);
+    at_n = at;
+    // This lane's page id of tile i + 1 is loaded while tile i is worked on (a page-table line is
+    // often no longer in L2 by the time it is needed).
     int nx_raw = -1;
     auto load_next = [&](long long t) {
       const long long g = g_begin + t;
-      at_n.seek(pre, g);
-      const int u = at_n.u;
-      const int lp = 2 * (int)(g - pre[u]) + half;
-      nx_raw = lp < p.max_pages ? __ldg(p.page_table + (size_t)urow[u] * p.max_pages + lp) : -1;
+      at_n.seek(pre, urow, ulen, g);
+      const int lp = 2 * (int)(g - at_n.first) + half;
+      nx_raw = lp < p.max_pages ? __ldg(p.page_table + (size_t)at_n.row * p.max_pages + lp) : -1;
     };
     if (n_tiles > 0) load_next(0);
     float sv[kPage];
     for (long long i = 0; i < n_tiles; ++i) {
       const long long g = g_begin + i;
-      at.seek(pre, g);
+      at.seek(pre, urow, ulen, g);
       const int u = at.u;
-      const int len_u = ulen[u], raw = nx_raw;  // raw: loaded during the previous tile
+      const int len_u = at.len, raw = nx_raw;  // raw: loaded during the previous tile
       if (i + 1 < n_tiles) load_next(i + 1);
-      const bool fresh = g == g_begin || g == pre[u];
-      const bool seg_end = g + 1 == g_end || g + 1 == pre[u + 1];
-      const int tt = (int)(g - pre[u]);
+      const bool fresh = g == g_begin || g == at.first;
+      const bool seg_end = g + 1 == g_end || g + 1 == at.next;
+      const int tt = (int)(g - at.first);
       const int nvalid = min(max(len_u - (2 * tt + half) * kPage, 0), kPage);
       const bool page_ok = nvalid > 0 && raw >= 0 && raw < p.num_pages;
       const int sb = (int)(i & 1);
@@ -764,7 +766,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         l_own = 0.f;
       }
       // ---- the scores of this lane's half of tile i ----
-      dead = __any_sync(0xffffffffu, dead || *(volatile int*)&tail->abort_ != 0);
+      dead = __any_sync(0xffffffffu, dead || ((i & 7) == 0 && *(volatile int*)&tail->abort_ != 0));
       wwait(&tail->s_full[sb], (uint32_t)((i >> 1) & 1));
       if (!dead) {
         // S = S_0 + S_1, the accumulators of the two score issuers (64 columns each)
