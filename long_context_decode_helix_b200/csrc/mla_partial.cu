@@ -64,10 +64,11 @@ constexpr int kTile = 2 * kPage;         // tokens per tile of the pair
 constexpr int kChunks = 9;               // 64-column chunks of a latent row
 constexpr int kSlot = 8192;              // one 64-column chunk of a page (64 rows x 128 B)
 constexpr int kQSlot = 2 * kSlot;        // score ring slot: two chunks of a page
-constexpr int kRingQ = 4;                // score-operand ring slots
+constexpr int kRingQ = 3;                // score-operand ring slots
 constexpr int kQSlotsPerTile = 5;        // chunks (0,1) (2,3) (4,5) (6,7) (8,-)
 constexpr int kVSlot = 2 * kSlot;        // value ring slot: 128 value columns of one page
-constexpr int kRingV = 3;                // value-operand ring slots
+constexpr int kRingV = 4;                // value-operand ring slots (a whole tile: the fourth slot
+                                         // of a tile would otherwise load only after P V took the first)
 constexpr int kQBytes = kChunks * kHc * 128;  // 72 KiB
 constexpr int kPBytes = 2 * kHc * 128;        // one tile's P: two 64-token K-chunks, 16 KiB
 constexpr uint32_t kOCol = 0, kSCol = 256, kTmemCols = 512;
@@ -919,38 +920,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         named_barrier_sync(1, kHeads);
         if (tail->flag) {  // merge every cluster's segment of this unit, for this CTA's heads
           __threadfence();
+          // segment c's record: the unit's first cluster used slot 1 unless its range started at
+          // the unit's first tile; every later cluster's range starts inside the unit (slot 0)
+          const int sl_lo = (range_begin(c_lo, W, Geff) >= pre[u]) ? 0 : 1;
+          auto rec_of = [&](int c) {
+            return p.seg + (((size_t)c * 2 + (c == c_lo ? sl_lo : 0)) * 2 + rank) * kRec;
+          };
           float Mm = -INFINITY;
-          for (int c = c_lo; c <= c_hi; ++c) {
-            const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
-            Mm = fmaxf(Mm, __ldcg(p.seg + (((size_t)c * 2 + sl) * 2 + rank) * kRec + kHc * kDV + hl));
-          }
+          for (int c = c_lo; c <= c_hi; ++c) Mm = fmaxf(Mm, __ldcg(rec_of(c) + kHc * kDV + hl));
           const float Mmu = Mm == -INFINITY ? 0.f : Mm;
           float Lm = 0.f, LBm = 0.f;
           for (int c = c_lo; c <= c_hi; ++c) {
-            const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
-            const float* rc = p.seg + (((size_t)c * 2 + sl) * 2 + rank) * kRec;
+            const float* rc = rec_of(c);
             const float w_ = fast_exp2(__ldcg(rc + kHc * kDV + hl) - Mmu);
             Lm += __ldcg(rc + kHc * kDV + kHc + hl) * w_;
             LBm += __ldcg(rc + kHc * kDV + 2 * kHc + hl) * w_;
           }
           const float invm = LBm > 0.f ? 1.f / LBm : 0.f;
-          // this thread merges its half of the head's 512 columns
+          // this thread merges its half of the head's 512 columns, 16 columns at a time
           for (int j = 0; j < 2; ++j) {
-            for (int cc = 0; cc < 128; cc += 4) {
-              const int col = 256 * j + 128 * half + cc;
-              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int c16 = 0; c16 < 128; c16 += 16) {
+              const int col = 256 * j + 128 * half + c16;
+              float4 acc[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
               for (int c = c_lo; c <= c_hi; ++c) {
-                const int sl = (range_begin(c, W, Geff) >= pre[u]) ? 0 : 1;
-                const float* rc = p.seg + (((size_t)c * 2 + sl) * 2 + rank) * kRec;
+                const float* rc = rec_of(c);
                 const float w_ = fast_exp2(__ldcg(rc + kHc * kDV + hl) - Mmu);
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(rc + hl * kDV + col));
-                acc.x += v.x * w_;
-                acc.y += v.y * w_;
-                acc.z += v.z * w_;
-                acc.w += v.w * w_;
+                const float4* src = reinterpret_cast<const float4*>(rc + hl * kDV + col);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float4 v = __ldcg(src + k);
+                  acc[k].x += v.x * w_;
+                  acc[k].y += v.y * w_;
+                  acc[k].z += v.z * w_;
+                  acc[k].w += v.w * w_;
+                }
               }
-              *reinterpret_cast<float4*>(p.o_part + orow * kDV + col) =
-                  make_float4(acc.x * invm, acc.y * invm, acc.z * invm, acc.w * invm);
+              float4* dst = reinterpret_cast<float4*>(p.o_part + orow * kDV + col);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_float4(acc[k].x * invm, acc[k].y * invm, acc[k].z * invm,
+                                     acc[k].w * invm);
             }
           }
           if (half == 0) p.lse[orow] = Lm > 0.f ? (Mm + log2f(Lm)) * kLn2 : -INFINITY;
