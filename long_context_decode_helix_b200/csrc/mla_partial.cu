@@ -33,7 +33,7 @@
 // Issue: a thread issuing a pair-wide tcgen05.mma is busy for longer than the tensor pipe needs
 // for these shapes, so three threads of CTA 0 issue: two take the first / second half of the
 // k-steps of every chunk into two score accumulators (the softmax adds them), the third issues
-// P V. They and the producers have the low warp ids; warps 4-7 are the softmax / epilogue warps.
+// P V. Warps 4-7 are the softmax / epilogue warps.
 // Softmax thread l reads TMEM lane l: lane l < 64 holds head l's scores of the first page of the
 // tile, lane 64 + l the same head's scores of the second page (the two-SM layout of an M =
 // 64-per-SM accumulator); the two threads of a head combine their row maxima through shared
@@ -72,10 +72,9 @@ constexpr int kRingV = 4;                // value-operand ring slots (a whole ti
 constexpr int kQBytes = kChunks * kHc * 128;  // 72 KiB
 constexpr int kPBytes = 2 * kHc * 128;        // one tile's P: two 64-token K-chunks, 16 KiB
 constexpr uint32_t kOCol = 0, kSCol = 256, kTmemCols = 512;
-// Warp roles. The MMA issuers and the producers take the low warp ids: when a softmax warp and one
-// of them are both ready on an SM sub-partition, the scheduler was measured to favour the older
-// warp, and a softmax warp with ready arithmetic otherwise starves a thread issuing tcgen05.mma.
-// Warps 4-7 are the softmax warps (warp w reads TMEM lanes 32 (w % 4) .. + 31).
+// Warp roles: the two score issuers, the P V issuer and the value producer on warps 0-3, the score
+// producer on warp 8, the softmax warps on 4-7 (warp w reads TMEM lanes 32 (w % 4) .. + 31). Each
+// of the three issuers shares its SM sub-partition with one softmax warp only.
 constexpr int kMmaWarp2 = 0, kMmaWarp = 1, kPvWarp = 2, kValueWarp = 3, kSoftmaxWarp0 = 4,
               kProducerWarp = 8;
 constexpr int kThreads = 9 * 32;
