@@ -748,7 +748,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       nx_raw = lp < p.max_pages ? __ldg(p.page_table + (size_t)at_n.row * p.max_pages + lp) : -1;
     };
     if (n_tiles > 0) load_next(0);
-    float sv[kPage];
     for (long long i = 0; i < n_tiles; ++i) {
       const long long g = g_begin + i;
       at.seek(pre, urow, ulen, g);
@@ -768,42 +767,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ---- the scores of this lane's half of tile i ----
       dead = __any_sync(0xffffffffu, dead || ((i & 7) == 0 && *(volatile int*)&tail->abort_ != 0));
       wwait(&tail->s_full[sb], (uint32_t)((i >> 1) & 1));
+      // S = S_0 + S_1 (the two score issuers' accumulators, 64 columns each), read twice in halves
+      // of 32 columns: once for the row maximum, once for the weights
+      const uint32_t sa = tl + kSCol + (uint32_t)sb * kTile;
+      const bool keep_all = nvalid == kPage && page_ok;
+      float mx = -INFINITY;
       if (!dead) {
-        // S = S_0 + S_1, the accumulators of the two score issuers (64 columns each)
         tc_fence_after();
-        const uint32_t sa = tl + kSCol + (uint32_t)sb * kTile;
-#pragma unroll
+#pragma unroll 1
         for (int h2 = 0; h2 < 2; ++h2) {
           float v0[32], v1[32];
           tmem_ld32_nowait(sa + 32 * h2, v0);
           tmem_ld32_nowait(sa + kTile / 2 + 32 * h2, v1);
           tmem_wait_ld();
+          float t[8];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) sv[32 * h2 + c] = v0[c] + v1[c];
+          for (int c = 0; c < 8; ++c) t[c] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            float x = v0[c] + v1[c];
+            if (!keep_all) x = (32 * h2 + c < nvalid && page_ok) ? x : -INFINITY;
+            t[c & 7] = fmaxf(t[c & 7], x);
+          }
+          mx = fmaxf(mx, fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])),
+                               fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7]))));
         }
-        tc_fence_before();
-      } else {
-#pragma unroll
-        for (int c = 0; c < kPage; ++c) sv[c] = 0.f;
       }
-      __syncwarp();
-      if (lane == 0) arrive_remote_relaxed(lead_s_empty + 8u * sb);  // S was read (wait::ld)
-      if (nvalid < kPage || !page_ok) {
-#pragma unroll
-        for (int c = 0; c < kPage; ++c) sv[c] = (c < nvalid && page_ok) ? sv[c] : -INFINITY;
-      }
-      float mx;
-      {  // tree reduction of this half's row maximum (raw scores; the scale is positive)
-        float t[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          t[c] = fmaxf(fmaxf(sv[c], sv[c + 16]), fmaxf(sv[c + 32], sv[c + 48]));
-#pragma unroll
-        for (int c = 0; c < 8; ++c) t[c] = fmaxf(t[c], t[c + 8]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) t[c] = fmaxf(t[c], t[c + 4]);
-        mx = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3])) * sl2;
-      }
+      mx *= sl2;
       // the head's maximum over both pages of the tile: the thread of the other half holds the rest
       // (double-buffered by tile parity: a buffer is rewritten only after the next exchange)
       tail->xmax[sb][lr] = mx;
@@ -818,23 +808,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float mb = m_new == -INFINITY ? 0.f : m_new;
       if (rescale) l_own *= fast_exp2(m_prev - mb);
       m_ref = m_new;
-      uint32_t pk[kPage / 2];
-      float ps[16];
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float p0 = fast_exp2(fmaf(sv[c], sl2, -mb)), p1 = fast_exp2(fmaf(sv[c + 1], sl2, -mb));
-        const float p2 = fast_exp2(fmaf(sv[c + 32], sl2, -mb));
-        const float p3 = fast_exp2(fmaf(sv[c + 33], sl2, -mb));
-        ps[c / 2] = (p0 + p1) + (p2 + p3);
-        pk[c / 2] = pack_bf16x2(p0, p1);
-        pk[16 + c / 2] = pack_bf16x2(p2, p3);
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) ps[c] += ps[c + 8];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
-      // O is normalised by the fp32 sum (the bf16-rounded weights differ from it by < 2^-9)
-      l_own += (ps[0] + ps[2]) + (ps[1] + ps[3]);
       // P(i) goes into buffer i % 2, last read by P V(i-2)
       if (i >= 2) wwait(&tail->p_empty[sb], (uint32_t)(((i - 2) >> 1) & 1));
       if (__any_sync(0xffffffffu, rescale) && !dead) {
@@ -855,15 +828,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       // this half's 64 weights of head hl: one 128-byte row of P's token chunk `half`, in the
       // 128-byte swizzled K-major layout the MMA reads (16-byte unit x of row r at x ^ (r % 8))
+      uint8_t* prow = p_s + (size_t)sb * kPBytes + (size_t)half * (kHc * 128) + hl * 128;
       if (!dead) {
-        uint8_t* prow = p_s + (size_t)sb * kPBytes + (size_t)half * (kHc * 128) + hl * 128;
+#pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
+          float v0[32], v1[32];
+          tmem_ld32_nowait(sa + 32 * h2, v0);
+          tmem_ld32_nowait(sa + kTile / 2 + 32 * h2, v1);
+          tmem_wait_ld();
+          uint32_t pk[16];
+          float ps[8];
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-          *reinterpret_cast<uint4*>(prow + ((x ^ (hl & 7)) << 4)) =
-              make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+          for (int c = 0; c < 32; c += 2) {
+            float x0 = v0[c] + v1[c], x1 = v0[c + 1] + v1[c + 1];
+            if (!keep_all) {
+              x0 = (32 * h2 + c < nvalid && page_ok) ? x0 : -INFINITY;
+              x1 = (32 * h2 + c + 1 < nvalid && page_ok) ? x1 : -INFINITY;
+            }
+            const float p0 = fast_exp2(fmaf(x0, sl2, -mb)), p1 = fast_exp2(fmaf(x1, sl2, -mb));
+            if (c < 16) ps[c / 2] = p0 + p1; else ps[(c - 16) / 2] += p0 + p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
+          // O is normalised by the fp32 sum (the bf16-rounded weights differ from it by < 2^-9)
+          l_own += (ps[0] + ps[2]) + (ps[1] + ps[3]);
+#pragma unroll
+          for (int xx = 0; xx < 4; ++xx)
+            *reinterpret_cast<uint4*>(prow + (((4 * h2 + xx) ^ (hl & 7)) << 4)) =
+                make_uint4(pk[4 * xx], pk[4 * xx + 1], pk[4 * xx + 2], pk[4 * xx + 3]);
+        }
       }
-      fence_proxy_async_smem();  // the generic-proxy P stores before the MMA's reads
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_remote_relaxed(lead_s_empty + 8u * sb);  // S was read (wait::ld)
+      fence_proxy_async_smem();  // the generic-proxy P stores before the MMA's reads
       __syncwarp();
       if (lane == 0) arrive_remote(lead_p_full + 8u * sb);
 
