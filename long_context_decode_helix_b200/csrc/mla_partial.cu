@@ -33,10 +33,11 @@
 // Issue: a thread issuing a pair-wide tcgen05.mma is busy for longer than the tensor pipe needs
 // for these shapes, so three threads of CTA 0 issue: two take the first / second half of the
 // k-steps of every chunk into two score accumulators (the softmax adds them), the third issues
-// P V. Warps 4-7 are the softmax / epilogue warps.
-// Softmax thread l reads TMEM lane l: lane l < 64 holds head l's scores of the first page of the
-// tile, lane 64 + l the same head's scores of the second page (the two-SM layout of an M =
-// 64-per-SM accumulator); the two threads of a head combine their row maxima through shared
+// P V. Warps 4-11 are the softmax / epilogue warps.
+// TMEM lane l holds head l's scores of the first page of the tile for l < 64, and lane 64 + l the
+// same head's scores of the second page (the two-SM layout of an M = 64-per-SM accumulator). Two
+// softmax threads read each lane, 32 columns each, once: the score buffer is released as soon as
+// that read completes, and the four threads of a head combine their row maxima through shared
 // memory. The tensor pipe computes the scores of tile i + 1 while the softmax works on tile i;
 // the scores and P each have two buffers. The reference maximum moves lazily (only when a row
 // maximum exceeds it by more than 8 in base-2 units), so weights stay below 2^8 and the TMEM
@@ -73,11 +74,12 @@ constexpr int kQBytes = kChunks * kHc * 128;  // 72 KiB
 constexpr int kPBytes = 2 * kHc * 128;        // one tile's P: two 64-token K-chunks, 16 KiB
 constexpr uint32_t kOCol = 0, kSCol = 256, kTmemCols = 512;
 // Warp roles: the two score issuers, the P V issuer and the value producer on warps 0-3, the score
-// producer on warp 8, the softmax warps on 4-7 (warp w reads TMEM lanes 32 (w % 4) .. + 31). Each
-// of the three issuers shares its SM sub-partition with one softmax warp only.
+// producer on warp 12, the softmax warps on 4-11 (warp w reads TMEM lanes 32 (w % 4) .. + 31; warps
+// w and w + 4 take the two 32-column halves of those lanes' scores).
 constexpr int kMmaWarp2 = 0, kMmaWarp = 1, kPvWarp = 2, kValueWarp = 3, kSoftmaxWarp0 = 4,
-              kProducerWarp = 8;
-constexpr int kThreads = 9 * 32;
+              kSoftmaxWarps = 8, kProducerWarp = 12;
+constexpr int kSoftThreads = kSoftmaxWarps * 32;
+constexpr int kThreads = 13 * 32;
 constexpr int kRec = kHc * (kDV + 3);    // floats per segment record (this CTA's heads)
 constexpr float kLazy = 8.f;             // base-2 headroom before the reference maximum moves
 constexpr int kPf = 2;                   // tiles whose pages are fetched into L2 ahead of the ring
@@ -89,14 +91,14 @@ struct MlaTail {
   uint64_t full_v[kRingV];   // the same for the value ring
   uint64_t empty_v[kRingV];
   uint64_t s_full[2];      // both: the scores of a tile are in TMEM (both score issuers)
-  uint64_t s_empty[2];     // CTA 0: the 4 softmax warps of each CTA read them
-  uint64_t p_full[2];      // CTA 0: the 4 softmax warps of each CTA wrote P (and rescaled O)
+  uint64_t s_empty[2];     // CTA 0: the 8 softmax warps of each CTA read them
+  uint64_t p_full[2];      // CTA 0: the 8 softmax warps of each CTA wrote P (and rescaled O)
   uint64_t p_empty[2];     // both: P V of the tile is done
   uint64_t q_full;         // CTA 0: its producer's arrival and both CTAs' q bytes
   uint64_t q_empty;        // both: the last score MMAs of a unit (both issuers) are done
   uint64_t mma_done;       // both: every MMA issued by the three issuers has completed
-  float xmax[2][kHeads];   // [tile parity][lane]: row maxima of the two token halves
-  float xl[kHeads];        // [lane]: row sums of the two halves at a segment end
+  float xmax[2][2][kHeads];  // [tile parity][column half][lane]: row maxima of a quarter tile
+  float xl[2][kHeads];       // [column half][lane]: row sums of a quarter at a segment end
   int pid[kPid][2];        // producer only: page ids (or -1) of the two pages of a tile
   uint32_t tmem_base;
   int flag;
@@ -343,8 +345,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tail->s_full[i], 2);  // the commits of both score issuers
-      mbar_init(&tail->s_empty[i], 8);  // the 4 softmax warps of each CTA
-      mbar_init(&tail->p_full[i], 8);
+      mbar_init(&tail->s_empty[i], 2 * kSoftmaxWarps);  // the softmax warps of both CTAs
+      mbar_init(&tail->p_full[i], 2 * kSoftmaxWarps);
       mbar_init(&tail->p_empty[i], 1);
     }
     mbar_init(&tail->q_full, 1);
@@ -719,17 +721,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (rank == 0 && lane == 0) tc_commit_pair(&tail->mma_done);
   } else {
     // ============================== softmax / epilogue warps =====================================
-    // Thread lr (= TMEM lane lr) holds local head hl = lr % 64 and the 64 tokens of page half =
-    // lr / 64 of each tile; the two threads of a head agree on its maximum through shared memory.
-    const int lr = tid - 32 * kSoftmaxWarp0;  // TMEM lane of this thread
+    // Thread (lr, ch) reads TMEM lane lr: local head hl = lr % 64, page half = lr / 64 of each tile,
+    // and of that page's 64 tokens the 32 in column half ch = 32 ch .. 32 ch + 31. The four threads
+    // of a head (two halves x two column halves) agree on its maximum through shared memory.
+    const int ch = (warp - kSoftmaxWarp0) >> 2;  // column half of the scores this warp reads
+    const int lr = 32 * (warp & 3) + lane;       // TMEM lane of this thread
     const int hl = lr & (kHc - 1);      // local head (row of this CTA's q)
     const int half = lr >> 6;           // which page of the tile this lane's scores belong to
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t lead_s_empty = map_rank(&tail->s_empty[0], 0);
     const uint32_t lead_p_full = map_rank(&tail->p_full[0], 0);
     const float sl2 = p.scale_log2;
-    float m_ref = -INFINITY;  // the head's reference maximum (base-2 logits), shared by both halves
-    float l_own = 0.f;        // running sum of this half's weights relative to m_ref
+    float m_ref = -INFINITY;  // the head's reference maximum (base-2 logits), shared by its threads
+    float l_own = 0.f;        // running sum of this thread's weights relative to m_ref
     bool dead = !active;
     auto wwait = [&](uint64_t* bar, uint32_t parity) {  // warp-uniform bounded wait
       if (dead) return;
@@ -764,41 +768,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         m_ref = -INFINITY;
         l_own = 0.f;
       }
-      // ---- the scores of this lane's half of tile i ----
+      // ---- this thread's 32 scores of tile i: S = S_0 + S_1 (the two score issuers' accumulators,
+      // 64 columns each), read once; the buffer is released as soon as the read has completed ----
       dead = __any_sync(0xffffffffu, dead || ((i & 7) == 0 && *(volatile int*)&tail->abort_ != 0));
       wwait(&tail->s_full[sb], (uint32_t)((i >> 1) & 1));
-      // S = S_0 + S_1 (the two score issuers' accumulators, 64 columns each), read twice in halves
-      // of 32 columns: once for the row maximum, once for the weights
-      const uint32_t sa = tl + kSCol + (uint32_t)sb * kTile;
+      const uint32_t sa = tl + kSCol + (uint32_t)sb * kTile + 32u * (uint32_t)ch;
       const bool keep_all = nvalid == kPage && page_ok;
+      float x[32];
       float mx = -INFINITY;
       if (!dead) {
         tc_fence_after();
-#pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-          float v0[32], v1[32];
-          tmem_ld32_nowait(sa + 32 * h2, v0);
-          tmem_ld32_nowait(sa + kTile / 2 + 32 * h2, v1);
-          tmem_wait_ld();
-          float t[8];
+        float v1[32];
+        tmem_ld32_nowait(sa, x);
+        tmem_ld32_nowait(sa + kTile / 2, v1);
+        tmem_wait_ld();
+        float t[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) t[c] = -INFINITY;
+        for (int c = 0; c < 8; ++c) t[c] = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float x = v0[c] + v1[c];
-            if (!keep_all) x = (32 * h2 + c < nvalid && page_ok) ? x : -INFINITY;
-            t[c & 7] = fmaxf(t[c & 7], x);
-          }
-          mx = fmaxf(mx, fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])),
-                               fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7]))));
+        for (int c = 0; c < 32; ++c) {
+          x[c] += v1[c];
+          if (!keep_all) x[c] = (32 * ch + c < nvalid && page_ok) ? x[c] : -INFINITY;
+          t[c & 7] = fmaxf(t[c & 7], x[c]);
         }
+        mx = fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])),
+                   fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = -INFINITY;
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_remote_relaxed(lead_s_empty + 8u * sb);  // S was read (wait::ld)
       mx *= sl2;
-      // the head's maximum over both pages of the tile: the thread of the other half holds the rest
+      // the head's maximum over the whole tile: the other three threads of the head hold the rest
       // (double-buffered by tile parity: a buffer is rewritten only after the next exchange)
-      tail->xmax[sb][lr] = mx;
-      named_barrier_sync(1, kHeads);
-      mx = fmaxf(mx, tail->xmax[sb][lr ^ 64]);
+      tail->xmax[sb][ch][lr] = mx;
+      named_barrier_sync(1, kSoftThreads);
+      mx = fmaxf(fmaxf(tail->xmax[sb][0][lr], tail->xmax[sb][1][lr]),
+                 fmaxf(tail->xmax[sb][0][lr ^ 64], tail->xmax[sb][1][lr ^ 64]));
       // ---- the reference maximum, lazily raised ----
       const float m_prev = m_ref;
       float m_new = m_prev;
@@ -810,58 +818,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       m_ref = m_new;
       // P(i) goes into buffer i % 2, last read by P V(i-2)
       if (i >= 2) wwait(&tail->p_empty[sb], (uint32_t)(((i - 2) >> 1) & 1));
+      // this thread's 32 weights of head hl: half of one 128-byte row of P's token chunk `half`, in
+      // the 128-byte swizzled K-major layout the MMA reads (16-byte unit x of row r at x ^ (r % 8))
+      uint8_t* prow = p_s + (size_t)sb * kPBytes + (size_t)half * (kHc * 128) + hl * 128;
+      if (!dead) {
+        uint32_t pk[16];
+        float ps[8];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = fast_exp2(fmaf(x[c], sl2, -mb)), p1 = fast_exp2(fmaf(x[c + 1], sl2, -mb));
+          if (c < 16) ps[c / 2] = p0 + p1; else ps[(c - 16) / 2] += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
+        // O is normalised by the fp32 sum (the bf16-rounded weights differ from it by < 2^-9)
+        l_own += (ps[0] + ps[2]) + (ps[1] + ps[3]);
+#pragma unroll
+        for (int xx = 0; xx < 4; ++xx)
+          *reinterpret_cast<uint4*>(prow + (((4 * ch + xx) ^ (hl & 7)) << 4)) =
+              make_uint4(pk[4 * xx], pk[4 * xx + 1], pk[4 * xx + 2], pk[4 * xx + 3]);
+      }
       if (__any_sync(0xffffffffu, rescale) && !dead) {
         // O holds the segment's tiles < i: wait for P V(i-1), then rescale the rows that moved
-        // (both threads of a head rescale their own lane). P V(i) cannot start before this
-        // warp's P is handed over, which comes after.
+        // (each thread of a head rescales its lane's columns 128 ch .. + 127), after P is written,
+        // when the scores no longer take registers. P V(i) cannot start before this warp's P is
+        // handed over, which comes after.
         wwait(&tail->p_empty[sb ^ 1], (uint32_t)(((i - 1) >> 1) & 1));
         const float alpha = rescale ? fast_exp2(m_prev - m_new) : 1.f;
         tc_fence_after();
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 0; c < 128; c += 32) {
           float o[32];
-          tmem_ld32(tl + kOCol + c, o);
+          tmem_ld32(tl + kOCol + 128 * ch + c, o);
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] *= alpha;
-          tmem_st32(tl + kOCol + c, o);
-        }
-        tc_fence_before();
-      }
-      // this half's 64 weights of head hl: one 128-byte row of P's token chunk `half`, in the
-      // 128-byte swizzled K-major layout the MMA reads (16-byte unit x of row r at x ^ (r % 8))
-      uint8_t* prow = p_s + (size_t)sb * kPBytes + (size_t)half * (kHc * 128) + hl * 128;
-      if (!dead) {
-#pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-          float v0[32], v1[32];
-          tmem_ld32_nowait(sa + 32 * h2, v0);
-          tmem_ld32_nowait(sa + kTile / 2 + 32 * h2, v1);
-          tmem_wait_ld();
-          uint32_t pk[16];
-          float ps[8];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float x0 = v0[c] + v1[c], x1 = v0[c + 1] + v1[c + 1];
-            if (!keep_all) {
-              x0 = (32 * h2 + c < nvalid && page_ok) ? x0 : -INFINITY;
-              x1 = (32 * h2 + c + 1 < nvalid && page_ok) ? x1 : -INFINITY;
-            }
-            const float p0 = fast_exp2(fmaf(x0, sl2, -mb)), p1 = fast_exp2(fmaf(x1, sl2, -mb));
-            if (c < 16) ps[c / 2] = p0 + p1; else ps[(c - 16) / 2] += p0 + p1;
-            pk[c / 2] = pack_bf16x2(p0, p1);
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
-          // O is normalised by the fp32 sum (the bf16-rounded weights differ from it by < 2^-9)
-          l_own += (ps[0] + ps[2]) + (ps[1] + ps[3]);
-#pragma unroll
-          for (int xx = 0; xx < 4; ++xx)
-            *reinterpret_cast<uint4*>(prow + (((4 * h2 + xx) ^ (hl & 7)) << 4)) =
-                make_uint4(pk[4 * xx], pk[4 * xx + 1], pk[4 * xx + 2], pk[4 * xx + 3]);
+          tmem_st32(tl + kOCol + 128 * ch + c, o);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_remote_relaxed(lead_s_empty + 8u * sb);  // S was read (wait::ld)
+      tc_fence_before();         // the O rescale before the MMA that reads it
       fence_proxy_async_smem();  // the generic-proxy P stores before the MMA's reads
       __syncwarp();
       if (lane == 0) arrive_remote(lead_p_full + 8u * sb);
@@ -870,10 +864,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ---- end of a segment: O is complete once P V(i) is ----
       wwait(&tail->p_empty[sb], (uint32_t)((i >> 1) & 1));
       tc_fence_after();
-      tail->xl[lr] = l_own;
-      named_barrier_sync(1, kHeads);
-      const float M = m_ref;  // the reference O and both sums are relative to
-      const float l_run = l_own + tail->xl[lr ^ 64];
+      tail->xl[ch][lr] = l_own;
+      named_barrier_sync(1, kSoftThreads);
+      const float M = m_ref;  // the reference O and all four sums are relative to
+      const float l_run = (tail->xl[0][lr] + tail->xl[1][lr]) + (tail->xl[0][lr ^ 64] + tail->xl[1][lr ^ 64]);
       const size_t orow = (size_t)urow[u] * kHeads + (size_t)rank * kHc + hl;
       const bool whole = g_begin <= pre[u] && g + 1 == pre[u + 1];
       float* rec = nullptr;
@@ -882,8 +876,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         rec = p.seg + (((size_t)pair * 2 + slot) * 2 + rank) * kRec;
       }
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      // TMEM lane lr, column block j: value columns [256 j + 128 half, + 128) of head hl
-      for (int j = 0; j < 2; ++j) {
+      // TMEM lane lr, column block j = ch: value columns [256 j + 128 half, + 128) of head hl
+      {
+        const int j = ch;
         for (int c = 0; c < 128; c += 32) {
           float o[32];
           if (!dead) tmem_ld32(tl + kOCol + j * 128 + c, o);
@@ -901,21 +896,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       if (whole) {
-        if (half == 0) p.lse[orow] = l_run > 0.f ? (M + log2f(l_run)) * kLn2 : -INFINITY;
+        if (half == 0 && ch == 0) p.lse[orow] = l_run > 0.f ? (M + log2f(l_run)) * kLn2 : -INFINITY;
       } else {
-        if (half == 0) {
+        if (half == 0 && ch == 0) {
           rec[kHc * kDV + hl] = M;
           rec[kHc * kDV + kHc + hl] = l_run;
           rec[kHc * kDV + 2 * kHc + hl] = l_run;
         }
         __threadfence();
-        named_barrier_sync(1, kHeads);
+        named_barrier_sync(1, kSoftThreads);
         const int c_lo = cta_of(pre[u], W, Geff), c_hi = cta_of((long long)pre[u + 1] - 1, W, Geff);
-        if (lr == 0) {
+        if (lr == 0 && ch == 0) {
           const int ticket = atomicAdd(&p.tickets[u * 2 + rank], 1);
           tail->flag = ticket == c_hi - c_lo;
         }
-        named_barrier_sync(1, kHeads);
+        named_barrier_sync(1, kSoftThreads);
         if (tail->flag) {  // merge every cluster's segment of this unit, for this CTA's heads
           __threadfence();
           // segment c's record: the unit's first cluster used slot 1 unless its range started at
@@ -935,8 +930,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             LBm += __ldcg(rc + kHc * kDV + 2 * kHc + hl) * w_;
           }
           const float invm = LBm > 0.f ? 1.f / LBm : 0.f;
-          // this thread merges its half of the head's 512 columns, 16 columns at a time
-          for (int j = 0; j < 2; ++j) {
+          // this thread merges its quarter of the head's 512 columns, 16 columns at a time
+          {
+            const int j = ch;
             for (int c16 = 0; c16 < 128; c16 += 16) {
               const int col = 256 * j + 128 * half + c16;
               float4 acc[4];
@@ -962,9 +958,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                      acc[k].w * invm);
             }
           }
-          if (half == 0) p.lse[orow] = Lm > 0.f ? (Mm + log2f(Lm)) * kLn2 : -INFINITY;
-          named_barrier_sync(1, kHeads);
-          if (lr == 0) p.tickets[u * 2 + rank] = 0;
+          if (half == 0 && ch == 0) p.lse[orow] = Lm > 0.f ? (Mm + log2f(Lm)) * kLn2 : -INFINITY;
+          named_barrier_sync(1, kSoftThreads);
+          if (lr == 0 && ch == 0) p.tickets[u * 2 + rank] = 0;
         }
       }
     }
