@@ -214,6 +214,17 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32])
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// Two IEEE fp32 additions / fused multiply-adds (round to nearest) in one instruction.
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%0, %1};\n mov.b64 rb, {%2, %3};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %4};\n"
+      " mov.b64 rc, {%5, %5};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -786,11 +797,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) t[c] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] += v1[c];
-          if (!keep_all) x[c] = (32 * ch + c < nvalid && page_ok) ? x[c] : -INFINITY;
-          t[c & 7] = fmaxf(t[c & 7], x[c]);
+        for (int c = 0; c < 32; c += 2) add2(x[c], x[c + 1], v1[c], v1[c + 1]);
+        if (!keep_all) {  // rare: the last, partial page of a shard, or a page id out of range
+          const int nv = page_ok ? nvalid - 32 * ch : 0;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = c < nv ? x[c] : -INFINITY;
         }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) t[c & 7] = fmaxf(t[c & 7], x[c]);
         mx = fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])),
                    fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
       } else {
@@ -826,14 +840,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float ps[8];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float p0 = fast_exp2(fmaf(x[c], sl2, -mb)), p1 = fast_exp2(fmaf(x[c + 1], sl2, -mb));
-          if (c < 16) ps[c / 2] = p0 + p1; else ps[(c - 16) / 2] += p0 + p1;
+          float z0, z1;
+          fma2(z0, z1, x[c], x[c + 1], sl2, -mb);
+          const float p0 = fast_exp2(z0), p1 = fast_exp2(z1);
+          if (c < 8) ps[c] = p0, ps[c + 1] = p1;
+          else add2(ps[c & 7], ps[(c & 7) + 1], p0, p1);
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
+        add2(ps[0], ps[1], ps[4], ps[5]);
+        add2(ps[2], ps[3], ps[6], ps[7]);
+        add2(ps[0], ps[1], ps[2], ps[3]);
         // O is normalised by the fp32 sum (the bf16-rounded weights differ from it by < 2^-9)
-        l_own += (ps[0] + ps[2]) + (ps[1] + ps[3]);
+        l_own += ps[0] + ps[1];
 #pragma unroll
         for (int xx = 0; xx < 4; ++xx)
           *reinterpret_cast<uint4*>(prow + (((4 * ch + xx) ^ (hl & 7)) << 4)) =
