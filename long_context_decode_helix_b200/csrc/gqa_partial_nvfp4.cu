@@ -117,6 +117,18 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// fma(a0, b, c), fma(a1, b, c) in one instruction (two IEEE round-to-nearest fused multiply-adds)
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %4};\n"
+      " mov.b64 rc, {%5, %5};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
   return pack_f16x2(bf16_lo_to_f32(v), bf16_hi_to_f32(v));
 }
@@ -333,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
     float mx0 = fmaxf(s[0][0], s[0][1]), mx1 = fmaxf(s[0][2], s[0][3]);
 #pragma unroll
     for (int n = 1; n < 8; ++n) {
-      mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
-      mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
+      mx0 = max3f(mx0, s[n][0], s[n][1]);
+      mx1 = max3f(mx1, s[n][2], s[n][3]);
     }
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
@@ -365,14 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1) gqa_partial_nvfp4_kernel(const Gq
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t pa[4];
-      pa[0] = pack_f16x2(fast_exp2(fmaf(s[2 * cc][0], sl2, -mu0)),
-                         fast_exp2(fmaf(s[2 * cc][1], sl2, -mu0)));
-      pa[1] = pack_f16x2(fast_exp2(fmaf(s[2 * cc][2], sl2, -mu1)),
-                         fast_exp2(fmaf(s[2 * cc][3], sl2, -mu1)));
-      pa[2] = pack_f16x2(fast_exp2(fmaf(s[2 * cc + 1][0], sl2, -mu0)),
-                         fast_exp2(fmaf(s[2 * cc + 1][1], sl2, -mu0)));
-      pa[3] = pack_f16x2(fast_exp2(fmaf(s[2 * cc + 1][2], sl2, -mu1)),
-                         fast_exp2(fmaf(s[2 * cc + 1][3], sl2, -mu1)));
+      float z[8];
+      fma2(z[0], z[1], s[2 * cc][0], s[2 * cc][1], sl2, -mu0);
+      fma2(z[2], z[3], s[2 * cc][2], s[2 * cc][3], sl2, -mu1);
+      fma2(z[4], z[5], s[2 * cc + 1][0], s[2 * cc + 1][1], sl2, -mu0);
+      fma2(z[6], z[7], s[2 * cc + 1][2], s[2 * cc + 1][3], sl2, -mu1);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pa[k] = pack_f16x2(fast_exp2(z[2 * k]), fast_exp2(z[2 * k + 1]));
       // token pairs (2t, 2t+1) and (2t+8, 2t+9) of the chunk; a pair row's 16-byte chunks are
       // stored XOR-swizzled by 2 (pair mod 4) = 2t, so a quarter-warp hits every bank once
       const int pa_ = 8 * cc + t4, pb_ = pa_ + 4;
