@@ -734,7 +734,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ============================== softmax / epilogue warps =====================================
     // Thread (lr, ch) reads TMEM lane lr: local head hl = lr % 64, page half = lr / 64 of each tile,
     // and of that page's 64 tokens the 32 in column half ch = 32 ch .. 32 ch + 31. The four threads
-    // of a head (two halves x two column halves) agree on its maximum through shared memory.
+    // of a head (two halves x two column halves) agree on its maximum through shared memory; those
+    // four warps have the same parity, so each tile's exchange waits on named barrier 1 (even warps)
+    // or 2 (odd warps), and only a segment end, where all eight meet, on barrier 3.
     const int ch = (warp - kSoftmaxWarp0) >> 2;  // column half of the scores this warp reads
     const int lr = 32 * (warp & 3) + lane;       // TMEM lane of this thread
     const int hl = lr & (kHc - 1);      // local head (row of this CTA's q)
@@ -818,7 +820,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // the head's maximum over the whole tile: the other three threads of the head hold the rest
       // (double-buffered by tile parity: a buffer is rewritten only after the next exchange)
       tail->xmax[sb][ch][lr] = mx;
-      named_barrier_sync(1, kSoftThreads);
+      // the four threads of a head are in warps w, w + 4, w ^ 2, (w ^ 2) + 4: warps of one parity
+      named_barrier_sync(1 + (warp & 1), kSoftThreads / 2);
       mx = fmaxf(fmaxf(tail->xmax[sb][0][lr], tail->xmax[sb][1][lr]),
                  fmaxf(tail->xmax[sb][0][lr ^ 64], tail->xmax[sb][1][lr ^ 64]));
       // ---- the reference maximum, lazily raised ----
@@ -883,7 +886,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       wwait(&tail->p_empty[sb], (uint32_t)((i >> 1) & 1));
       tc_fence_after();
       tail->xl[ch][lr] = l_own;
-      named_barrier_sync(1, kSoftThreads);
+      named_barrier_sync(3, kSoftThreads);
       const float M = m_ref;  // the reference O and all four sums are relative to
       const float l_run = (tail->xl[0][lr] + tail->xl[1][lr]) + (tail->xl[0][lr ^ 64] + tail->xl[1][lr ^ 64]);
       const size_t orow = (size_t)urow[u] * kHeads + (size_t)rank * kHc + hl;
@@ -922,13 +925,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           rec[kHc * kDV + 2 * kHc + hl] = l_run;
         }
         __threadfence();
-        named_barrier_sync(1, kSoftThreads);
+        named_barrier_sync(3, kSoftThreads);
         const int c_lo = cta_of(pre[u], W, Geff), c_hi = cta_of((long long)pre[u + 1] - 1, W, Geff);
         if (lr == 0 && ch == 0) {
           const int ticket = atomicAdd(&p.tickets[u * 2 + rank], 1);
           tail->flag = ticket == c_hi - c_lo;
         }
-        named_barrier_sync(1, kSoftThreads);
+        named_barrier_sync(3, kSoftThreads);
         if (tail->flag) {  // merge every cluster's segment of this unit, for this CTA's heads
           __threadfence();
           // segment c's record: the unit's first cluster used slot 1 unless its range started at
@@ -977,7 +980,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
           if (half == 0 && ch == 0) p.lse[orow] = Lm > 0.f ? (Mm + log2f(Lm)) * kLn2 : -INFINITY;
-          named_barrier_sync(1, kSoftThreads);
+          named_barrier_sync(3, kSoftThreads);
           if (lr == 0 && ch == 0) p.tickets[u * 2 + rank] = 0;
         }
       }
