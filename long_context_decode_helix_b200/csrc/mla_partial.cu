@@ -14,7 +14,7 @@
 // of one SM, and q (128 x 576 bf16) alone is 144 KiB. A cluster of two CTAs therefore splits the
 // HEADS: CTA r owns heads [64 r, 64 r + 64), holds their q (72 KiB) in shared memory and their O
 // (64 x 512 fp32) in 256 TMEM columns, and every MMA is a pair-wide tcgen05.mma.cta_group::2
-// issued by one thread of CTA 0, in which each SM computes the rows of its own heads:
+// issued by a thread of CTA 0, in which each SM computes the rows of its own heads:
 //   * scores S = q C^T per 128-token tile (two pages; CTA r loads page r of the two), M = 128
 //     heads (64 per SM), N = 128 tokens (each CTA supplies the 64 rows of its page as its half of
 //     B), K = 576 in 36 steps: each SM ends with the complete scores of its 64 heads for all 128
@@ -24,10 +24,10 @@
 //     128 tokens. P is written to shared memory by the softmax warps (the A operand, K-major);
 //     V is read again from L2 into the value ring (MN-major), two 64-column chunks x 64 tokens.
 // Operands stream through two rings of 16 KiB shared-memory slots, one per operand, each filled by
-// a producer warp in both CTAs: the score ring takes this CTA's page of each tile as five slots of
-// two 64-column chunks (one 3-D TMA box each; the fifth holds chunk 8 and zeros), the value ring
-// takes, per column block j and page, this CTA's two 64-column chunks of that page (read again,
-// from L2). Every TMA load of either CTA completes on CTA 0's barrier of its slot; the MMAs'
+// a producer warp in both CTAs: the score ring (3 slots) takes this CTA's page of each tile as five
+// slots of two 64-column chunks (one 3-D TMA box each; the fifth holds chunk 8 and zeros), the
+// value ring (4 slots, a whole tile) takes, per column block j and page, this CTA's two 64-column
+// chunks of that page (read again, from L2). Every TMA load of either CTA completes on CTA 0's barrier of its slot; the MMAs'
 // commits reach both CTAs (tcgen05.commit multicast). No TMA load uses cluster multicast.
 //
 // Issue: a thread issuing a pair-wide tcgen05.mma is busy for longer than the tensor pipe needs
