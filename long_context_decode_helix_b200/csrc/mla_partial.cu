@@ -97,7 +97,7 @@ struct MlaTail {
   uint64_t q_full;         // CTA 0: its producer's arrival and both CTAs' q bytes
   uint64_t q_empty;        // both: the last score MMAs of a unit (both issuers) are done
   uint64_t mma_done;       // both: every MMA issued by the three issuers has completed
-  float xmax[2][2][kHeads];  // [tile parity][column half][lane]: row maxima of a quarter tile
+  float xmax[2][kHeads][2];  // [tile parity][lane][column half]: row maxima of a quarter tile
   float xl[2][kHeads];       // [column half][lane]: row sums of a quarter at a segment end
   int pid[kPid][2];        // producer only: page ids (or -1) of the two pages of a tile
   uint32_t tmem_base;
@@ -225,6 +225,12 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
       " mov.b64 rc, {%5, %5};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
       : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -297,8 +303,8 @@ struct UnitCursor {
     len = ulen[u];
   }
   // moves to the unit of tile g (g never decreases); true when the unit changed
-  __device__ __forceinline__ bool seek(const int* pre, const int* urow, const int* ulen,
-                                       long long g) {
+  template <class G>
+  __device__ __forceinline__ bool seek(const int* pre, const int* urow, const int* ulen, G g) {
     if (g < next) return false;
     do {
       ++u;
@@ -758,22 +764,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // This lane's page id of tile i + 1 is loaded while tile i is worked on (a page-table line is
     // often no longer in L2 by the time it is needed).
     int nx_raw = -1;
-    auto load_next = [&](long long t) {
-      const long long g = g_begin + t;
-      at_n.seek(pre, urow, ulen, g);
-      const int lp = 2 * (int)(g - at_n.first) + half;
-      nx_raw = lp < p.max_pages ? __ldg(p.page_table + (size_t)at_n.row * p.max_pages + lp) : -1;
+    // tile indices fit in 32 bits (a launch's tiles are counted in int)
+    const int gb = (int)g_begin, ge = (int)g_end, nt = (int)n_tiles;
+    const int* pt_row = p.page_table + (size_t)at_n.row * p.max_pages;  // at_n's page-table row
+    auto load_next = [&](int t) {
+      const int g = gb + t;
+      if (at_n.seek(pre, urow, ulen, g)) pt_row = p.page_table + (size_t)at_n.row * p.max_pages;
+      const int lp = 2 * (g - at_n.first) + half;
+      nx_raw = lp < p.max_pages ? __ldg(pt_row + lp) : -1;
     };
-    if (n_tiles > 0) load_next(0);
-    for (long long i = 0; i < n_tiles; ++i) {
-      const long long g = g_begin + i;
+    if (nt > 0) load_next(0);
+    for (int i = 0; i < nt; ++i) {
+      const int g = gb + i;
       at.seek(pre, urow, ulen, g);
       const int u = at.u;
       const int len_u = at.len, raw = nx_raw;  // raw: loaded during the previous tile
-      if (i + 1 < n_tiles) load_next(i + 1);
-      const bool fresh = g == g_begin || g == at.first;
-      const bool seg_end = g + 1 == g_end || g + 1 == at.next;
-      const int tt = (int)(g - at.first);
+      if (i + 1 < nt) load_next(i + 1);
+      const bool fresh = g == gb || g == at.first;
+      const bool seg_end = g + 1 == ge || g + 1 == at.next;
+      const int tt = g - at.first;
       const int nvalid = min(max(len_u - (2 * tt + half) * kPage, 0), kPage);
       const bool page_ok = nvalid > 0 && raw >= 0 && raw < p.num_pages;
       const int sb = (int)(i & 1);
@@ -795,9 +804,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_ld32_nowait(sa, x);
         tmem_ld32_nowait(sa + kTile / 2, v1);
         tmem_wait_ld();
-        float t[8];
+        float t[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) t[c] = -INFINITY;
+        for (int c = 0; c < 4; ++c) t[c] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 32; c += 2) add2(x[c], x[c + 1], v1[c], v1[c + 1]);
         if (!keep_all) {  // rare: the last, partial page of a shard, or a page id out of range
@@ -806,9 +815,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 32; ++c) x[c] = c < nv ? x[c] : -INFINITY;
         }
 #pragma unroll
-        for (int c = 0; c < 32; ++c) t[c & 7] = fmaxf(t[c & 7], x[c]);
-        mx = fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])),
-                   fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
+        for (int c = 0; c < 32; c += 2) t[(c >> 1) & 3] = max3f(t[(c >> 1) & 3], x[c], x[c + 1]);
+        mx = max3f(max3f(t[0], t[1], t[2]), t[3], t[3]);
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) x[c] = -INFINITY;
@@ -819,11 +827,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mx *= sl2;
       // the head's maximum over the whole tile: the other three threads of the head hold the rest
       // (double-buffered by tile parity: a buffer is rewritten only after the next exchange)
-      tail->xmax[sb][ch][lr] = mx;
+      tail->xmax[sb][lr][ch] = mx;
       // the four threads of a head are in warps w, w + 4, w ^ 2, (w ^ 2) + 4: warps of one parity
       named_barrier_sync(1 + (warp & 1), kSoftThreads / 2);
-      mx = fmaxf(fmaxf(tail->xmax[sb][0][lr], tail->xmax[sb][1][lr]),
-                 fmaxf(tail->xmax[sb][0][lr ^ 64], tail->xmax[sb][1][lr ^ 64]));
+      {
+        const float2 a = *reinterpret_cast<const float2*>(&tail->xmax[sb][lr][0]);
+        const float2 b = *reinterpret_cast<const float2*>(&tail->xmax[sb][lr ^ 64][0]);
+        mx = max3f(max3f(a.x, a.y, b.x), b.y, b.y);
+      }
       // ---- the reference maximum, lazily raised ----
       const float m_prev = m_ref;
       float m_new = m_prev;
