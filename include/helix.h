@@ -163,7 +163,7 @@ helix_status helix_attn_workspace_size(const helix_kv_cache* cache, int32_t num_
  * A shard with no tokens gives O_s = 0 and lse = -inf.
  * GQA: num_q_heads % H == 0 and num_q_heads / H <= 16. MLA: num_q_heads == 128.
  * Work is enqueued on `stream` as one kernel launch, except for MLA batches with more (request,
- * shard) units than one launch keeps in shared memory (about 1,850 on a B200): those run as
+ * shard) units than one launch keeps in shared memory (about 570 on a B200): those run as
  * consecutive launches over request ranges, sharing the workspace, with the same results.
  * HELIX_ERR_CAPACITY only if one request's units do not fit.
  */
