@@ -54,6 +54,9 @@ constexpr int kPage = 64;
 constexpr int kRows = 16;
 constexpr int kWarps = 8;  // one page each; each owns ring slots 2 w and 2 w + 1
 constexpr int kThreads = kWarps * 32;
+// the fixed-order merge of the warps' O and the segment flush's (row, column) split of the threads
+// are written for exactly this count
+static_assert(kWarps == 8 && kThreads == 16 * 16, "segment flush written for eight warps");
 constexpr int kNStage = 2 * kWarps;
 constexpr int kKcBytes = kPage * kD / 2;   // 4096
 constexpr int kKsBytes = kPage * kD / 16;  // 512

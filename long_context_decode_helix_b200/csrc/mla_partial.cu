@@ -80,6 +80,10 @@ constexpr int kMmaWarp2 = 0, kMmaWarp = 1, kPvWarp = 2, kValueWarp = 3, kSoftmax
               kSoftmaxWarps = 8, kProducerWarp = 12;
 constexpr int kSoftThreads = kSoftmaxWarps * 32;
 constexpr int kThreads = 13 * 32;
+// two softmax warps per TMEM lane quarter, one per 32-column half of the page's scores
+static_assert(kSoftmaxWarps == 8 && kProducerWarp == kSoftmaxWarp0 + kSoftmaxWarps &&
+                  kThreads == (kProducerWarp + 1) * 32,
+              "the softmax's column split is written for two warps per lane quarter");
 constexpr int kRec = kHc * (kDV + 3);    // floats per segment record (this CTA's heads)
 constexpr float kLazy = 8.f;             // base-2 headroom before the reference maximum moves
 constexpr int kPf = 2;                   // tiles whose pages are fetched into L2 ahead of the ring
