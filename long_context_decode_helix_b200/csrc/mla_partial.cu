@@ -813,7 +813,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 4; ++c) t[c] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 32; c += 2) add2(x[c], x[c + 1], v1[c], v1[c + 1]);
-        if (!keep_all) {  // rare: the last, partial page of a shard, or a page id out of range
+        // rare: the last, partial page of a shard, or a page id out of range
+        if (__builtin_expect(!keep_all, 0)) {
           const int nv = page_ok ? nvalid - 32 * ch : 0;
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c] = c < nv ? x[c] : -INFINITY;
@@ -875,7 +876,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(prow + (((4 * ch + xx) ^ (hl & 7)) << 4)) =
               make_uint4(pk[4 * xx], pk[4 * xx + 1], pk[4 * xx + 2], pk[4 * xx + 3]);
       }
-      if (__any_sync(0xffffffffu, rescale) && !dead) {
+      if (__builtin_expect(__any_sync(0xffffffffu, rescale) && !dead, 0)) {
         // O holds the segment's tiles < i: wait for P V(i-1), then rescale the rows that moved
         // (each thread of a head rescales its lane's columns 128 ch .. + 127), after P is written,
         // when the scores no longer take registers. P V(i) cannot start before this warp's P is
@@ -896,7 +897,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) arrive_remote(lead_p_full + 8u * sb);
 
-      if (!seg_end) continue;
+      if (__builtin_expect(!seg_end, 1)) continue;
       // ---- end of a segment: O is complete once P V(i) is ----
       wwait(&tail->p_empty[sb], (uint32_t)((i >> 1) & 1));
       tc_fence_after();
