@@ -101,7 +101,8 @@ struct MlaTail {
   uint64_t q_full;         // CTA 0: its producer's arrival and both CTAs' q bytes
   uint64_t q_empty;        // both: the last score MMAs of a unit (both issuers) are done
   uint64_t mma_done;       // both: every MMA issued by the three issuers has completed
-  float xmax[2][kHeads][2];  // [tile parity][lane][column half]: row maxima of a quarter tile
+  // [tile parity][lane][column half]: row maxima of a quarter tile (read as 8-byte pairs)
+  alignas(8) float xmax[2][kHeads][2];
   float xl[2][kHeads];       // [column half][lane]: row sums of a quarter at a segment end
   int pid[kPid][2];        // producer only: page ids (or -1) of the two pages of a tile
   uint32_t tmem_base;
